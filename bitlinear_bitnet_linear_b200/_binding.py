@@ -1,0 +1,245 @@
+"""ctypes binding for libbitnet.so: argument marshalling only.
+
+Every function here has the name of the C entry point it calls
+(include/bitnet.h), takes torch CUDA tensors, passes their device pointers
+and the current CUDA stream, and raises BitnetError on a non-OK status.
+No arithmetic of the method happens in Python; there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitnet.so")
+
+OK = 0
+STATUS_NAMES = {0: "OK", 1: "ERR_NULL", 2: "ERR_SHAPE", 3: "ERR_ALIGN", 4: "ERR_DTYPE",
+                5: "ERR_UNSUPPORTED", 6: "ERR_CUDA", 7: "ERR_TIMEOUT", 8: "ERR_WORKSPACE",
+                9: "ERR_VALUE"}
+F32, BF16 = 0, 1
+PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
+
+# every symbol declared in include/bitnet.h
+EXPORTS = ("bitnet_workspace_bytes", "bitnet_quant_weights_workspace_bytes", "bitnet_workspace_init",
+           "bitnet_get_error", "bitnet_status_str", "bitnet_quant_weights", "bitnet_ternarise",
+           "bitnet_pack", "bitnet_unpack", "bitnet_quant_act", "bitnet_linear", "bitnet_linear_ex",
+           "bitnet_linear_q", "bitnet_set_wait_limit_us", "bitnet_watchdog_selftest")
+
+
+class BitnetError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)} ({status_str(status)})")
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbitnet.so (built in-tree by build.py); raise if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"libbitnet.so not built ({LIB_PATH}); run bitlinear_bitnet_linear_b200.build.build()")
+    L = ctypes.CDLL(LIB_PATH)
+    P, I64, I32, U32, F, SZ = (ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint32,
+                               ctypes.c_float, ctypes.c_size_t)
+    sig = {
+        "bitnet_workspace_bytes": ([I64, I64, I64], SZ),
+        "bitnet_quant_weights_workspace_bytes": ([I64, I64], SZ),
+        "bitnet_workspace_init": ([P, SZ, P], I32),
+        "bitnet_get_error": ([P, P], I32),
+        "bitnet_status_str": ([I32], ctypes.c_char_p),
+        "bitnet_quant_weights": ([P, I64, I64, F, P, P, P, SZ, P], I32),
+        "bitnet_ternarise": ([P, I64, I64, P, F, P, P], I32),
+        "bitnet_pack": ([P, I64, I64, P, P, P], I32),
+        "bitnet_unpack": ([P, I64, I64, P, P, P], I32),
+        "bitnet_quant_act": ([P, I32, I64, I64, P, F, P, P, P, P], I32),
+        "bitnet_linear": ([P, I32, I64, I64, P, I64, P, P, F, P, I32, P, SZ, P], I32),
+        "bitnet_linear_ex": ([P, I32, I64, I64, P, I64, P, P, F, P, I32, P, SZ, I32, P], I32),
+        "bitnet_linear_q": ([P, P, P, I64, I64, P, I64, P, P, I32, P, P, SZ, I32, P], I32),
+        "bitnet_set_wait_limit_us": ([U32], I32),
+        "bitnet_watchdog_selftest": ([P, SZ, U32, P], I32),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(L, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = L
+    return L
+
+
+def status_str(s: int) -> str:
+    try:
+        return lib().bitnet_status_str(int(s)).decode()
+    except Exception:  # pragma: no cover - only when the library is absent
+        return "?"
+
+
+def _check(st: int, what: str) -> None:
+    if st != OK:
+        raise BitnetError(st, what)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _xdtype(t) -> int:
+    if t.dtype == torch.float32:
+        return F32
+    if t.dtype == torch.bfloat16:
+        return BF16
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _ydtype(d) -> int:
+    return {torch.float32: F32, torch.bfloat16: BF16}[d]
+
+
+# --------------------------------------------------------------------------
+# workspace
+# --------------------------------------------------------------------------
+
+def bitnet_workspace_bytes(M: int, K: int, N: int) -> int:
+    return int(lib().bitnet_workspace_bytes(M, K, N))
+
+
+def bitnet_quant_weights_workspace_bytes(N: int, K: int) -> int:
+    return int(lib().bitnet_quant_weights_workspace_bytes(N, K))
+
+
+def new_workspace(nbytes: int, device=None) -> torch.Tensor:
+    """A zeroed device buffer usable as a workspace (torch blocks are 512-byte aligned)."""
+    n = max(256, (int(nbytes) + 255) // 256 * 256)
+    return torch.zeros(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def bitnet_workspace_init(ws: torch.Tensor, stream=None) -> None:
+    _check(lib().bitnet_workspace_init(_ptr(ws), ws.numel(), _stream(stream)), "bitnet_workspace_init")
+
+
+def bitnet_get_error(ws: torch.Tensor, stream=None) -> int:
+    """Synchronise and return (and clear) the workspace's device status."""
+    return int(lib().bitnet_get_error(_ptr(ws), _stream(stream)))
+
+
+def bitnet_set_wait_limit_us(limit_us: int) -> None:
+    _check(lib().bitnet_set_wait_limit_us(int(limit_us)), "bitnet_set_wait_limit_us")
+
+
+def bitnet_watchdog_selftest(ws: torch.Tensor, limit_us: int, stream=None) -> None:
+    _check(lib().bitnet_watchdog_selftest(_ptr(ws), ws.numel(), int(limit_us), _stream(stream)),
+           "bitnet_watchdog_selftest")
+
+
+# --------------------------------------------------------------------------
+# weight preparation
+# --------------------------------------------------------------------------
+
+def bitnet_quant_weights(W: torch.Tensor, eps: float = 1e-8, Wq: torch.Tensor | None = None,
+                         gamma: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                         want_wq: bool = True, stream=None):
+    """Returns (Wq int8 [N, K] or None, gamma float32 [1]) on W's device."""
+    N, K = W.shape
+    if want_wq and Wq is None:
+        Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    if ws is None:
+        ws = new_workspace(bitnet_quant_weights_workspace_bytes(N, K), W.device)
+    _check(lib().bitnet_quant_weights(_ptr(W), N, K, float(eps), _ptr(Wq) if want_wq else None, _ptr(gamma),
+                                      _ptr(ws), ws.numel(), _stream(stream)), "bitnet_quant_weights")
+    return Wq, gamma
+
+
+def bitnet_ternarise(W: torch.Tensor, gamma: torch.Tensor, eps: float = 1e-8, Wq=None, stream=None):
+    N, K = W.shape
+    if Wq is None:
+        Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    _check(lib().bitnet_ternarise(_ptr(W), N, K, _ptr(gamma), float(eps), _ptr(Wq), _stream(stream)),
+           "bitnet_ternarise")
+    return Wq
+
+
+def bitnet_pack(Wq: torch.Tensor, Wp=None, n_invalid=None, stream=None):
+    N, K = Wq.shape
+    if Wp is None:
+        Wp = torch.empty((N, K // 4), dtype=torch.uint8, device=Wq.device)
+    _check(lib().bitnet_pack(_ptr(Wq), N, K, _ptr(Wp), _ptr(n_invalid), _stream(stream)), "bitnet_pack")
+    return Wp
+
+
+def bitnet_unpack(Wp: torch.Tensor, K: int, Wq=None, n_invalid=None, stream=None):
+    N = Wp.shape[0]
+    if Wq is None:
+        Wq = torch.empty((N, K), dtype=torch.int8, device=Wp.device)
+    _check(lib().bitnet_unpack(_ptr(Wp), N, K, _ptr(Wq), _ptr(n_invalid), _stream(stream)), "bitnet_unpack")
+    return Wq
+
+
+# --------------------------------------------------------------------------
+# per-call path
+# --------------------------------------------------------------------------
+
+def bitnet_quant_act(x: torch.Tensor, rms_gain: torch.Tensor | None = None, rms_eps: float = 1e-5,
+                     xq=None, x_scale=None, x_sum=None, want_sum: bool = True, stream=None):
+    M, K = x.shape
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if x_scale is None:
+        x_scale = torch.empty(M, dtype=torch.float32, device=x.device)
+    if want_sum and x_sum is None:
+        x_sum = torch.empty(M, dtype=torch.int32, device=x.device)
+    _check(lib().bitnet_quant_act(_ptr(x), _xdtype(x), M, K, _ptr(rms_gain), float(rms_eps), _ptr(xq),
+                                  _ptr(x_scale), _ptr(x_sum) if want_sum else None, _stream(stream)),
+           "bitnet_quant_act")
+    return xq, x_scale, (x_sum if want_sum else None)
+
+
+def bitnet_linear(x: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N: int | None = None,
+                  rms_gain: torch.Tensor | None = None, rms_eps: float = 1e-5, y=None,
+                  y_dtype=torch.bfloat16, ws=None, path: int = PATH_AUTO, stream=None):
+    M, K = x.shape
+    N = Wp.shape[0] if N is None else N
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=x.device)
+    if ws is None:
+        ws = new_workspace(bitnet_workspace_bytes(M, K, N), x.device)
+    _check(lib().bitnet_linear_ex(_ptr(x), _xdtype(x), M, K, _ptr(Wp), N, _ptr(gamma), _ptr(rms_gain),
+                                  float(rms_eps), _ptr(y), _ydtype(y.dtype), _ptr(ws), ws.numel(), int(path),
+                                  _stream(stream)), "bitnet_linear")
+    return y
+
+
+def bitnet_linear_q(xq: torch.Tensor, x_scale: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor,
+                    x_sum: torch.Tensor | None = None, y=None, y_dtype=torch.float32, want_y: bool = True,
+                    acc=None, want_acc: bool = False, ws=None, path: int = PATH_AUTO, stream=None):
+    M, K = xq.shape
+    N = Wp.shape[0]
+    if want_y and y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=xq.device)
+    if want_acc and acc is None:
+        acc = torch.empty((M, N), dtype=torch.int32, device=xq.device)
+    if ws is None:
+        ws = new_workspace(bitnet_workspace_bytes(M, K, N), xq.device)
+    _check(lib().bitnet_linear_q(_ptr(xq), _ptr(x_scale), _ptr(x_sum), M, K, _ptr(Wp), N, _ptr(gamma),
+                                 _ptr(y) if want_y else None, _ydtype(y.dtype) if want_y else F32,
+                                 _ptr(acc) if want_acc else None, _ptr(ws), ws.numel(), int(path),
+                                 _stream(stream)), "bitnet_linear_q")
+    return y, acc

@@ -1,0 +1,524 @@
+// bitnet.cu -- the C ABI of libbitnet.so (declared in include/bitnet.h):
+// argument validation, path selection and kernel launches.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <mutex>
+
+#include "act.cuh"
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "gemv.cuh"
+#include "weights.cuh"
+
+using namespace bitnet;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kGemvMaxM = 4;
+constexpr size_t kWsHeader = sizeof(WsHeader);
+
+std::atomic<uint64_t> g_limit_ns{2000000000ull};
+
+struct DeviceInfo {
+  bool init = false;
+  bool ok = false;
+  int sms = 0;
+  int max_smem_optin = 0;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_mu;
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bitnet_status cuda_status(cudaError_t e) { return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA; }
+
+bitnet_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return BITNET_ERR_UNSUPPORTED;
+  }
+  if (dev < 0 || dev >= kMaxDevices) return BITNET_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.init) {
+    d.init = true;
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&d.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    cudaGetLastError();
+    d.ok = (major == 10 && minor == 0 && d.sms > 0);
+  }
+  if (!d.ok) return BITNET_ERR_UNSUPPORTED;
+  *out = &d;
+  return BITNET_OK;
+}
+
+bitnet_status get_encoder() {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_encode != nullptr) return BITNET_OK;
+  cudaDriverEntryPointQueryResult q;
+  void* fn = nullptr;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || fn == nullptr) {
+    cudaGetLastError();
+    return BITNET_ERR_CUDA;
+  }
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return BITNET_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+bitnet_status check_shape(int64_t M, int64_t K, int64_t N) {
+  if (M < 1 || N < 1 || K < 16 || (K % 16) != 0) return BITNET_ERR_SHAPE;
+  const int64_t lim = (int64_t(1) << 31) - 1;
+  if (M > lim || N > lim || K > lim) return BITNET_ERR_SHAPE;
+  if (N * K >= (int64_t(1) << 39) || M * K >= (int64_t(1) << 39) || M * N >= (int64_t(1) << 39))
+    return BITNET_ERR_SHAPE;
+  return BITNET_OK;
+}
+
+// Launch with programmatic stream serialisation allowed.
+template <typename Kern, typename... Args>
+cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+template <typename Kern>
+cudaError_t allow_smem(Kern kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+}
+
+int elementwise_grid(int64_t work, const DeviceInfo* d) {
+  const int64_t g = (work + 255) / 256;
+  const int64_t cap = static_cast<int64_t>(d->sms) * 16;
+  return static_cast<int>(g < 1 ? 1 : (g > cap ? cap : g));
+}
+
+// Workspace carve-up for the linear calls.
+struct LinearWs {
+  uint32_t* status;
+  int8_t* xq;
+  float* scale;
+  int32_t* sum;
+};
+size_t linear_ws_bytes(int64_t M, int64_t K) {
+  return kWsHeader + round_up(static_cast<size_t>(M * K), 256) + 2 * round_up(static_cast<size_t>(M) * 4, 256);
+}
+LinearWs carve(void* ws, int64_t M, int64_t K) {
+  LinearWs w;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  w.status = reinterpret_cast<uint32_t*>(b);
+  b += kWsHeader;
+  w.xq = reinterpret_cast<int8_t*>(b);
+  b += round_up(static_cast<size_t>(M * K), 256);
+  w.scale = reinterpret_cast<float*>(b);
+  b += round_up(static_cast<size_t>(M) * 4, 256);
+  w.sum = reinterpret_cast<int32_t*>(b);
+  return w;
+}
+
+// ---------------------------------------------------------------------------
+// GEMV launch planning.
+// ---------------------------------------------------------------------------
+struct GemvPlan {
+  int MT, R, grid, smem;
+  GemvParams p;
+};
+
+bitnet_status plan_gemv(const DeviceInfo* d, int64_t M, int64_t K, int64_t N, GemvPlan& pl) {
+  if (M > kGemvMaxM) return BITNET_ERR_UNSUPPORTED;
+  pl.MT = M <= 1 ? 1 : (M <= 2 ? 2 : 4);
+  pl.R = K <= 4096 ? 4 : (K <= 8192 ? 2 : 1);
+  if (pl.MT == 4 && pl.R == 4) pl.R = 2;
+  GemvParams& p = pl.p;
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(K);
+  p.N = static_cast<int>(N);
+  p.Kp = static_cast<int>(round_up(static_cast<size_t>(K), 64));
+  p.bulk = (K % 64 == 0) ? 1 : 0;
+  p.wrow = p.bulk ? static_cast<int>(K / 4) : p.Kp / 4;
+  const int grid = static_cast<int>(N < d->sms ? N : d->sms);
+  pl.grid = grid;
+  p.rows_base = static_cast<int>(N / grid);
+  p.rows_extra = static_cast<int>(N % grid);
+  const int rows_cta = p.rows_base + (p.rows_extra ? 1 : 0);
+  const int xbytes = pl.MT * p.Kp;
+  // Prefer a footprint that lets the next call's CTAs co-reside (PDL
+  // overlap); grow only when one stage would not fit.
+  const int budget_soft = 112 * 1024;
+  const int budget_hard = d->max_smem_optin;
+  int stage_rows = kGvWarps * pl.R;
+  if (stage_rows > rows_cta) stage_rows = rows_cta;
+  const int stage_bytes = stage_rows * p.wrow;
+  const int nst = (rows_cta + stage_rows - 1) / stage_rows;
+  int room = budget_soft - kGvHeader - xbytes;
+  if (room < 2 * stage_bytes) room = budget_hard - kGvHeader - xbytes;
+  int stages = room / stage_bytes;
+  if (stages > kGvMaxStages) stages = kGvMaxStages;
+  if (stages > nst) stages = nst;
+  if (stages < 1) return BITNET_ERR_UNSUPPORTED;
+  p.stage_rows = stage_rows;
+  p.stages = stages;
+  pl.smem = kGvHeader + xbytes + stages * stage_bytes;
+  if (pl.smem > budget_hard) return BITNET_ERR_UNSUPPORTED;
+  return BITNET_OK;
+}
+
+template <int MT, int R, bool FUSED>
+cudaError_t run_gemv_t(const GemvPlan& pl, cudaStream_t st) {
+  auto k = gemv_kernel<MT, R, FUSED>;
+  cudaError_t e = allow_smem(k, pl.smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k, dim3(pl.grid), dim3(kGvThreads), pl.smem, st, pl.p);
+}
+
+template <bool FUSED>
+cudaError_t run_gemv(const GemvPlan& pl, cudaStream_t st) {
+  switch (pl.MT * 10 + pl.R) {
+    case 14: return run_gemv_t<1, 4, FUSED>(pl, st);
+    case 12: return run_gemv_t<1, 2, FUSED>(pl, st);
+    case 11: return run_gemv_t<1, 1, FUSED>(pl, st);
+    case 22: return run_gemv_t<2, 2, FUSED>(pl, st);
+    case 24: return run_gemv_t<2, 4, FUSED>(pl, st);
+    case 21: return run_gemv_t<2, 1, FUSED>(pl, st);
+    case 42: return run_gemv_t<4, 2, FUSED>(pl, st);
+    case 41: return run_gemv_t<4, 1, FUSED>(pl, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Tensor-core GEMM launch.
+// ---------------------------------------------------------------------------
+template <int BM, int STAGES>
+cudaError_t run_tc_t(const int8_t* xq, const TcParams& p, cudaStream_t st) {
+  CUtensorMap map;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.K), static_cast<cuuint64_t>(p.M)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.K)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcBK), static_cast<cuuint32_t>(BM)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(xq), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  auto k = tc_gemm_kernel<BM, STAGES>;
+  constexpr int smem = tc_smem_bytes<BM, STAGES>();
+  cudaError_t e = allow_smem(k, smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid((p.N + kTcBN - 1) / kTcBN, (p.M + BM - 1) / BM);
+  return launch_pdl(k, grid, dim3(kTcThreads), smem, st, map, p);
+}
+
+cudaError_t run_tc(const int8_t* xq, const TcParams& p, cudaStream_t st) {
+  if (p.M <= 16) return run_tc_t<16, 8>(xq, p, st);
+  if (p.M <= 32) return run_tc_t<32, 8>(xq, p, st);
+  if (p.M <= 64) return run_tc_t<64, 8>(xq, p, st);
+  if (p.M <= 128) return run_tc_t<128, 6>(xq, p, st);
+  return run_tc_t<256, 4>(xq, p, st);
+}
+
+bitnet_status launch_result(cudaError_t e) {
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return BITNET_ERR_CUDA;
+  }
+  e = cudaGetLastError();
+  return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
+}
+
+}  // namespace
+
+// ===========================================================================
+// Exported C ABI
+// ===========================================================================
+extern "C" {
+
+size_t bitnet_workspace_bytes(int64_t M, int64_t K, int64_t N) {
+  (void)N;
+  if (M < 1 || K < 1) return kWsHeader;
+  return linear_ws_bytes(M, K);
+}
+
+size_t bitnet_quant_weights_workspace_bytes(int64_t N, int64_t K) {
+  const int64_t n = N * K;
+  int64_t blocks = (n + kAbsMaxPerBlock - 1) / kAbsMaxPerBlock;
+  const int64_t want = 148 * 8;
+  if (blocks < want) blocks = want;
+  return kWsHeader + static_cast<size_t>(blocks) * kAbsBins * sizeof(uint64_t);
+}
+
+bitnet_status bitnet_workspace_init(void* ws, size_t ws_bytes, bitnet_stream_t stream) {
+  if (ws == nullptr) return BITNET_ERR_NULL;
+  if (ws_bytes < kWsHeader || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return BITNET_ERR_WORKSPACE;
+  return cuda_status(cudaMemsetAsync(ws, 0, kWsHeader, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+bitnet_status bitnet_get_error(void* ws, bitnet_stream_t stream) {
+  if (ws == nullptr) return BITNET_ERR_NULL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t h[2] = {0, 0};
+  if (cudaMemcpyAsync(h, ws, sizeof h, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return BITNET_ERR_CUDA;
+  }
+  if (h[0] != 0) {
+    if (cudaMemsetAsync(ws, 0, sizeof h, st) != cudaSuccess || cudaStreamSynchronize(st) != cudaSuccess) {
+      cudaGetLastError();
+      return BITNET_ERR_CUDA;
+    }
+  }
+  return static_cast<bitnet_status>(h[0]);
+}
+
+const char* bitnet_status_str(bitnet_status s) {
+  switch (s) {
+    case BITNET_OK: return "ok";
+    case BITNET_ERR_NULL: return "null pointer";
+    case BITNET_ERR_SHAPE: return "invalid shape (M, N >= 1; K a positive multiple of 16)";
+    case BITNET_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case BITNET_ERR_DTYPE: return "unknown dtype";
+    case BITNET_ERR_UNSUPPORTED: return "unsupported (needs an sm_100 device, or the forced path cannot run)";
+    case BITNET_ERR_CUDA: return "CUDA runtime error";
+    case BITNET_ERR_TIMEOUT: return "device wait timed out";
+    case BITNET_ERR_WORKSPACE: return "workspace missing, too small or misaligned";
+    case BITNET_ERR_VALUE: return "invalid ternary value or code";
+  }
+  return "unknown status";
+}
+
+bitnet_status bitnet_set_wait_limit_us(uint32_t limit_us) {
+  if (limit_us == 0) return BITNET_ERR_SHAPE;
+  g_limit_ns.store(static_cast<uint64_t>(limit_us) * 1000ull);
+  return BITNET_OK;
+}
+
+bitnet_status bitnet_quant_weights(const float* W, int64_t N, int64_t K, float eps, int8_t* Wq, float* gamma,
+                                   void* ws, size_t ws_bytes, bitnet_stream_t stream) {
+  if (W == nullptr || gamma == nullptr || ws == nullptr) return BITNET_ERR_NULL;
+  if (check_shape(1, K, N) != BITNET_OK) return BITNET_ERR_SHAPE;
+  if (!aligned16(W) || (Wq != nullptr && !aligned16(Wq))) return BITNET_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < bitnet_quant_weights_workspace_bytes(N, K))
+    return BITNET_ERR_WORKSPACE;
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t n = N * K;
+  int64_t blocks = (n + kAbsMaxPerBlock - 1) / kAbsMaxPerBlock;
+  const int64_t want = static_cast<int64_t>(d->sms) * 8;
+  if (blocks < want) blocks = want;
+  const int64_t cap = static_cast<int64_t>((ws_bytes - kWsHeader) / (kAbsBins * sizeof(uint64_t)));
+  if (blocks > cap) blocks = cap;
+  int64_t per_block = (n + blocks - 1) / blocks;
+  per_block = (per_block + 15) / 16 * 16;          // keep float4 alignment
+  if (per_block > kAbsMaxPerBlock) return BITNET_ERR_WORKSPACE;
+  blocks = (n + per_block - 1) / per_block;
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  uint64_t* partial = reinterpret_cast<uint64_t*>(static_cast<uint8_t*>(ws) + kWsHeader);
+  absmean_partial_kernel<<<static_cast<unsigned>(blocks), kAbsThreads, 0, st>>>(W, n, per_block, partial, status);
+  absmean_finalize_kernel<<<1, 32, 0, st>>>(partial, static_cast<int>(blocks), n, gamma);
+  if (Wq != nullptr) {
+    ternarise_kernel<<<elementwise_grid(n / 4, d), 256, 0, st>>>(W, n / 4, gamma, eps, Wq);
+  }
+  return launch_result(cudaSuccess);
+}
+
+bitnet_status bitnet_ternarise(const float* W, int64_t N, int64_t K, const float* gamma, float eps, int8_t* Wq,
+                               bitnet_stream_t stream) {
+  if (W == nullptr || gamma == nullptr || Wq == nullptr) return BITNET_ERR_NULL;
+  if (check_shape(1, K, N) != BITNET_OK) return BITNET_ERR_SHAPE;
+  if (!aligned16(W) || !aligned16(Wq)) return BITNET_ERR_ALIGN;
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  const int64_t n = N * K;
+  ternarise_kernel<<<elementwise_grid(n / 4, d), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(W, n / 4, gamma,
+                                                                                                     eps, Wq);
+  return launch_result(cudaSuccess);
+}
+
+bitnet_status bitnet_pack(const int8_t* Wq, int64_t N, int64_t K, uint8_t* Wp, uint32_t* n_invalid,
+                          bitnet_stream_t stream) {
+  if (Wq == nullptr || Wp == nullptr) return BITNET_ERR_NULL;
+  if (check_shape(1, K, N) != BITNET_OK) return BITNET_ERR_SHAPE;
+  if (!aligned16(Wq) || !aligned16(Wp)) return BITNET_ERR_ALIGN;
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t groups = N * K / 16;
+  pack_kernel<<<elementwise_grid(groups, d), 256, 0, st>>>(Wq, groups, reinterpret_cast<uint32_t*>(Wp), n_invalid);
+  stream_fence_kernel<<<1, 32, 0, st>>>();
+  return launch_result(cudaSuccess);
+}
+
+bitnet_status bitnet_unpack(const uint8_t* Wp, int64_t N, int64_t K, int8_t* Wq, uint32_t* n_invalid,
+                            bitnet_stream_t stream) {
+  if (Wq == nullptr || Wp == nullptr) return BITNET_ERR_NULL;
+  if (check_shape(1, K, N) != BITNET_OK) return BITNET_ERR_SHAPE;
+  if (!aligned16(Wq) || !aligned16(Wp)) return BITNET_ERR_ALIGN;
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  const int64_t groups = N * K / 16;
+  unpack_kernel<<<elementwise_grid(groups, d), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint32_t*>(Wp), groups, Wq, n_invalid);
+  return launch_result(cudaSuccess);
+}
+
+bitnet_status bitnet_quant_act(const void* x, int x_dtype, int64_t M, int64_t K, const float* rms_gain,
+                               float rms_eps, int8_t* xq, float* x_scale, int32_t* x_sum, bitnet_stream_t stream) {
+  if (x == nullptr || xq == nullptr || x_scale == nullptr) return BITNET_ERR_NULL;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (check_shape(M, K, 1) != BITNET_OK) return BITNET_ERR_SHAPE;
+  if (!aligned16(x) || !aligned16(xq) || (rms_gain != nullptr && !aligned16(rms_gain))) return BITNET_ERR_ALIGN;
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  cudaError_t e = launch_pdl(quant_act_kernel, dim3(static_cast<unsigned>(M)), dim3(kActThreads), 0,
+                             reinterpret_cast<cudaStream_t>(stream), x, x_dtype, static_cast<int>(K), rms_gain,
+                             rms_eps, xq, x_scale, x_sum);
+  return launch_result(e);
+}
+
+static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in, const float* scale_in,
+                                 const int32_t* sum_in, int64_t M, int64_t K, const uint8_t* Wp, int64_t N,
+                                 const float* gamma, const float* rms_gain, float rms_eps, void* y, int y_dtype,
+                                 int32_t* acc, void* ws, size_t ws_bytes, int path, cudaStream_t st) {
+  if (Wp == nullptr || gamma == nullptr || ws == nullptr) return BITNET_ERR_NULL;
+  if (y == nullptr && acc == nullptr) return BITNET_ERR_NULL;
+  if (y != nullptr && y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  bitnet_status s = check_shape(M, K, N);
+  if (s != BITNET_OK) return s;
+  if (!aligned16(Wp) || (y != nullptr && !aligned16(y)) || (acc != nullptr && !aligned16(acc)) ||
+      (rms_gain != nullptr && !aligned16(rms_gain)))
+    return BITNET_ERR_ALIGN;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < kWsHeader) return BITNET_ERR_WORKSPACE;
+  if (path != BITNET_PATH_AUTO && path != BITNET_PATH_GEMV && path != BITNET_PATH_TC) return BITNET_ERR_UNSUPPORTED;
+  DeviceInfo* d;
+  s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  uint32_t* status = static_cast<uint32_t*>(ws);
+  const uint64_t limit = g_limit_ns.load();
+
+  GemvPlan gp;
+  bool gemv_ok = plan_gemv(d, M, K, N, gp) == BITNET_OK;
+  if (path == BITNET_PATH_GEMV && !gemv_ok) return BITNET_ERR_UNSUPPORTED;
+  const bool use_gemv = (path == BITNET_PATH_GEMV) || (path == BITNET_PATH_AUTO && gemv_ok);
+
+  if (use_gemv) {
+    GemvParams& p = gp.p;
+    p.x = x;
+    p.x_dtype = x_dtype;
+    p.gain = rms_gain;
+    p.rms_eps = rms_eps;
+    p.xq = xq_in;
+    p.x_scale = scale_in;
+    p.Wp = Wp;
+    p.gamma = gamma;
+    p.y = y;
+    p.y_dtype = y_dtype;
+    p.acc = acc;
+    p.limit_ns = limit;
+    p.status = status;
+    cudaError_t e = (x != nullptr) ? run_gemv<true>(gp, st) : run_gemv<false>(gp, st);
+    return launch_result(e);
+  }
+
+  // Tensor-core path: quantised activations must sit in memory for TMA.
+  s = get_encoder();
+  if (s != BITNET_OK) return s;
+  const int8_t* xq = xq_in;
+  const float* scale = scale_in;
+  const int32_t* sum = sum_in;
+  if (x != nullptr) {
+    if (ws_bytes < linear_ws_bytes(M, K)) return BITNET_ERR_WORKSPACE;
+    LinearWs w = carve(ws, M, K);
+    cudaError_t e = launch_pdl(quant_act_kernel, dim3(static_cast<unsigned>(M)), dim3(kActThreads), 0, st, x,
+                               x_dtype, static_cast<int>(K), rms_gain, rms_eps, w.xq, w.scale, w.sum);
+    if (e != cudaSuccess) return launch_result(e);
+    xq = w.xq;
+    scale = w.scale;
+    sum = w.sum;
+  } else if (sum == nullptr) {
+    if (ws_bytes < linear_ws_bytes(M, K)) return BITNET_ERR_WORKSPACE;
+    LinearWs w = carve(ws, M, K);
+    cudaError_t e = launch_pdl(xq_rowsum_kernel, dim3(static_cast<unsigned>(M)), dim3(kActThreads), 0, st, xq,
+                               static_cast<int>(K), w.sum);
+    if (e != cudaSuccess) return launch_result(e);
+    sum = w.sum;
+  }
+  TcParams p;
+  p.Wp = Wp;
+  p.gamma = gamma;
+  p.x_scale = scale;
+  p.x_sum = sum;
+  p.y = y;
+  p.y_dtype = y_dtype;
+  p.acc = acc;
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(K);
+  p.N = static_cast<int>(N);
+  p.KB = static_cast<int>((K + kTcBK - 1) / kTcBK);
+  p.wvec = (K % 64 == 0) ? 1 : 0;
+  p.limit_ns = limit;
+  p.status = status;
+  return launch_result(run_tc(xq, p, st));
+}
+
+bitnet_status bitnet_linear_ex(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t* Wp, int64_t N,
+                               const float* gamma, const float* rms_gain, float rms_eps, void* y, int y_dtype,
+                               void* ws, size_t ws_bytes, int path, bitnet_stream_t stream) {
+  if (x == nullptr || y == nullptr) return BITNET_ERR_NULL;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (!aligned16(x)) return BITNET_ERR_ALIGN;
+  return linear_impl(x, x_dtype, nullptr, nullptr, nullptr, M, K, Wp, N, gamma, rms_gain, rms_eps, y, y_dtype,
+                     nullptr, ws, ws_bytes, path, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitnet_status bitnet_linear(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t* Wp, int64_t N,
+                            const float* gamma, const float* rms_gain, float rms_eps, void* y, int y_dtype, void* ws,
+                            size_t ws_bytes, bitnet_stream_t stream) {
+  return bitnet_linear_ex(x, x_dtype, M, K, Wp, N, gamma, rms_gain, rms_eps, y, y_dtype, ws, ws_bytes,
+                          BITNET_PATH_AUTO, stream);
+}
+
+bitnet_status bitnet_linear_q(const int8_t* xq, const float* x_scale, const int32_t* x_sum, int64_t M, int64_t K,
+                              const uint8_t* Wp, int64_t N, const float* gamma, void* y, int y_dtype, int32_t* acc,
+                              void* ws, size_t ws_bytes, int path, bitnet_stream_t stream) {
+  if (xq == nullptr || x_scale == nullptr) return BITNET_ERR_NULL;
+  if (!aligned16(xq)) return BITNET_ERR_ALIGN;
+  return linear_impl(nullptr, BITNET_F32, xq, x_scale, x_sum, M, K, Wp, N, gamma, nullptr, 0.0f, y, y_dtype, acc, ws,
+                     ws_bytes, path, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitnet_status bitnet_watchdog_selftest(void* ws, size_t ws_bytes, uint32_t limit_us, bitnet_stream_t stream) {
+  if (ws == nullptr) return BITNET_ERR_NULL;
+  if (ws_bytes < kWsHeader || (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return BITNET_ERR_WORKSPACE;
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_us) * 1000ull, static_cast<uint32_t*>(ws));
+  return launch_result(cudaSuccess);
+}
+
+}  // extern "C"

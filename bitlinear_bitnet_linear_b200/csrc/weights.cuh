@@ -1,0 +1,232 @@
+// weights.cuh -- offline weight preparation: exact absmean scale, ternary
+// rounding, 2-bit pack and unpack.
+//
+// Absmean ternarisation follows "Key Technologies Enabling the BitNET
+// Family" (Advanced Quantization Methodologies: absmean ternary weights)
+// and "BitNet / Ternary / Binary -- Les LLMs 1-bit" (BitLinear forward:
+// beta = mean|w|, clamp(round(w / (beta + 1e-8)), -1, 1)).  The 2-bit
+// layout is this library's (2 bits per weight: "BitNet Technical Notes").
+#pragma once
+
+#include "common.cuh"
+
+namespace bitnet {
+
+// ---------------------------------------------------------------------------
+// Exact sum of |W|.
+//
+// Every finite binary32 magnitude is an integer multiple of 2^-149:
+//   |w| = M * 2^(E - 150),  M = 2^23 + mantissa (E >= 1) or mantissa with
+//   E := 1 (subnormal).
+// Split E = 16b + r.  Bin b accumulates M << r (< 2^39) in a uint64; a block
+// handles at most 2^24 elements, so a bin cannot overflow.  The per-block
+// bins are integers, so the final total does not depend on the order of
+// accumulation: gamma is deterministic for any launch shape.
+// ---------------------------------------------------------------------------
+constexpr int kAbsThreads = 256;
+constexpr int kAbsBins = 16;
+constexpr int64_t kAbsMaxPerBlock = int64_t(1) << 24;
+
+__device__ __forceinline__ void abs_bin_add(uint64_t* my_bins /* stride kAbsThreads */, float v, bool& bad) {
+  uint32_t bits = __float_as_uint(v) & 0x7fffffffu;
+  uint32_t e = bits >> 23;
+  uint32_t m = bits & 0x7fffffu;
+  if (e == 255u) { bad = true; return; }
+  if (e == 0u) {
+    if (m == 0u) return;
+    e = 1u;
+  } else {
+    m |= 0x800000u;
+  }
+  my_bins[(e >> 4) * kAbsThreads] += static_cast<uint64_t>(m) << (e & 15u);
+}
+
+__global__ void __launch_bounds__(kAbsThreads) absmean_partial_kernel(const float* __restrict__ W, int64_t n,
+                                                                      int64_t per_block,
+                                                                      uint64_t* __restrict__ partial,
+                                                                      uint32_t* status) {
+  __shared__ uint64_t bins[kAbsBins * kAbsThreads];
+  const int tid = threadIdx.x;
+  for (int b = 0; b < kAbsBins; ++b) bins[b * kAbsThreads + tid] = 0;
+  uint64_t* mine = bins + tid;
+  bool bad = false;
+
+  const int64_t b0 = static_cast<int64_t>(blockIdx.x) * per_block;
+  const int64_t b1 = min(n, b0 + per_block);
+  // per_block and n are multiples of 16, W is 16-byte aligned: float4 loads.
+  const float4* W4 = reinterpret_cast<const float4*>(W);
+  for (int64_t i = b0 / 4 + tid; i < b1 / 4; i += kAbsThreads) {
+    float4 v = __ldg(W4 + i);
+    abs_bin_add(mine, v.x, bad);
+    abs_bin_add(mine, v.y, bad);
+    abs_bin_add(mine, v.z, bad);
+    abs_bin_add(mine, v.w, bad);
+  }
+  if (bad) record_error(status, BITNET_ERR_VALUE, 0x101u);
+  __syncthreads();
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int b = warp; b < kAbsBins; b += kAbsThreads / 32) {
+    uint64_t s = 0;
+    for (int t = lane; t < kAbsThreads; t += 32) s += bins[b * kAbsThreads + t];
+    s = warp_sum<unsigned long long>(s);
+    if (lane == 0) partial[static_cast<int64_t>(blockIdx.x) * kAbsBins + b] = s;
+  }
+}
+
+// One warp: sum the per-block bins, assemble the exact total in a 384-bit
+// integer (units of 2^-150), round it once to binary64, divide by n in
+// binary64 and round to binary32.
+__global__ void absmean_finalize_kernel(const uint64_t* __restrict__ partial, int nblocks, int64_t n,
+                                        float* __restrict__ gamma_out) {
+  __shared__ unsigned long long lo_s[kAbsBins], hi_s[kAbsBins];
+  const int lane = threadIdx.x;
+  if (lane < kAbsBins) {
+    unsigned __int128 s = 0;
+    for (int b = 0; b < nblocks; ++b) s += partial[static_cast<int64_t>(b) * kAbsBins + lane];
+    lo_s[lane] = static_cast<unsigned long long>(s);
+    hi_s[lane] = static_cast<unsigned long long>(s >> 64);
+  }
+  __syncwarp();
+  if (lane != 0) return;
+
+  uint64_t limb[6] = {0, 0, 0, 0, 0, 0};
+  for (int b = 0; b < kAbsBins; ++b) {
+    // add (hi:lo) << 16b
+    const int sh = 16 * b, li = sh >> 6, off = sh & 63;
+    const uint64_t lo = lo_s[b], hi = hi_s[b];
+    uint64_t w[3];
+    w[0] = lo << off;
+    w[1] = (off ? (lo >> (64 - off)) : 0ull) | (hi << off);
+    w[2] = off ? (hi >> (64 - off)) : 0ull;
+    uint64_t carry = 0;
+    for (int t = 0; li + t < 6; ++t) {
+      const uint64_t add = (t < 3 ? w[t] : 0ull);
+      const uint64_t s1 = limb[li + t] + add;
+      const uint64_t c1 = s1 < add ? 1ull : 0ull;
+      const uint64_t s2 = s1 + carry;
+      const uint64_t c2 = s2 < carry ? 1ull : 0ull;
+      limb[li + t] = s2;
+      carry = c1 + c2;
+      if (t >= 2 && carry == 0) break;
+    }
+  }
+  int top = -1;
+  for (int i = 5; i >= 0; --i)
+    if (limb[i]) { top = i; break; }
+  double total;
+  if (top < 0) {
+    total = 0.0;
+  } else {
+    const int p = 64 * top + (63 - __clzll(static_cast<long long>(limb[top])));
+    if (p < 64) {
+      total = scalbn(__ull2double_rn(limb[0]), -150);
+    } else {
+      const int lob = p - 63;          // keep bits [lob, lob + 63]
+      const int li = lob >> 6, off = lob & 63;
+      uint64_t word = limb[li] >> off;
+      if (off && li + 1 < 6) word |= limb[li + 1] << (64 - off);
+      bool sticky = (off != 0) && ((limb[li] & ((1ull << off) - 1ull)) != 0);
+      for (int i = 0; i < li; ++i) sticky = sticky || (limb[i] != 0);
+      if (sticky) word |= 1ull;
+      total = scalbn(__ull2double_rn(word), lob - 150);
+    }
+  }
+  const double mean = __ddiv_rn(total, static_cast<double>(n));
+  *gamma_out = __double2float_rn(mean);
+}
+
+// ---------------------------------------------------------------------------
+// Ternary rounding: q = clamp(rint(w / (gamma + eps)), -1, 1), binary32.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int8_t ternary_of(float w, float d) {
+  const float r = rintf(__fdiv_rn(w, d));
+  return r >= 1.0f ? int8_t(1) : (r <= -1.0f ? int8_t(-1) : int8_t(0));
+}
+
+__global__ void __launch_bounds__(256) ternarise_kernel(const float* __restrict__ W, int64_t n4,
+                                                        const float* __restrict__ gamma, float eps,
+                                                        int8_t* __restrict__ Wq) {
+  const float d = __fadd_rn(*gamma, eps);
+  const float4* W4 = reinterpret_cast<const float4*>(W);
+  char4* Q4 = reinterpret_cast<char4*>(Wq);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 v = __ldg(W4 + i);
+    char4 q;
+    q.x = ternary_of(v.x, d);
+    q.y = ternary_of(v.y, d);
+    q.z = ternary_of(v.z, d);
+    q.w = ternary_of(v.w, d);
+    Q4[i] = q;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// 2-bit pack / unpack.  One thread per 16-weight group (one 32-bit word):
+// weight k = 16g + 4s + j at bits [8j + 2s, 8j + 2s + 1], code = q + 1.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) pack_kernel(const int8_t* __restrict__ Wq, int64_t ngroups,
+                                                   uint32_t* __restrict__ Wp, uint32_t* n_invalid) {
+  uint32_t bad = 0;
+  const uint4* Q = reinterpret_cast<const uint4*>(Wq);
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < ngroups;
+       g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 v = __ldg(Q + g);
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};   // in[s] byte j = q[16g + 4s + j]
+    uint32_t word = 0;
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int q = static_cast<int8_t>((in[s] >> (8 * j)) & 0xffu);
+        uint32_t c;
+        if (q >= -1 && q <= 1) {
+          c = static_cast<uint32_t>(q + 1);
+        } else {
+          c = 3u;
+          ++bad;
+        }
+        word |= c << (8 * j + 2 * s);
+      }
+    }
+    Wp[g] = word;
+  }
+  if (n_invalid != nullptr && bad) atomicAdd(n_invalid, bad);
+}
+
+__global__ void __launch_bounds__(256) unpack_kernel(const uint32_t* __restrict__ Wp, int64_t ngroups,
+                                                     int8_t* __restrict__ Wq, uint32_t* n_invalid) {
+  uint32_t bad = 0;
+  uint4* Q = reinterpret_cast<uint4*>(Wq);
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < ngroups;
+       g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t word = __ldg(Wp + g);
+    uint32_t out[4];
+#pragma unroll
+    for (int s = 0; s < 4; ++s) {
+      uint32_t o = 0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t c = (word >> (8 * j + 2 * s)) & 3u;
+        int q;
+        if (c == 3u) {
+          q = 0;
+          ++bad;
+        } else {
+          q = static_cast<int>(c) - 1;
+        }
+        o |= (static_cast<uint32_t>(q) & 0xffu) << (8 * j);
+      }
+      out[s] = o;
+    }
+    Q[g] = make_uint4(out[0], out[1], out[2], out[3]);
+  }
+  if (n_invalid != nullptr && bad) atomicAdd(n_invalid, bad);
+}
+
+// Empty kernel launched WITHOUT programmatic serialisation after calls that
+// write weights: a following GEMV may read weights before its dependency
+// wait, so the weight writer must be fully complete first.
+__global__ void stream_fence_kernel() {}
+
+}  // namespace bitnet

@@ -137,10 +137,12 @@ void orc_ternarise(const float *W, int64_t n, float gamma, float eps, int8_t *Wq
     for (int64_t i = 0; i < n; ++i) {
         float t = W[i] / d;
         float r = rintf(t);
+        /* r is integer-valued, so clamping to [-1, 1] is a three-way test; */
+        /* a NaN quotient (0/0 when gamma + eps == 0) compares false: 0.     */
         int8_t q;
-        if (r > 1.0f) q = 1;
-        else if (r < -1.0f) q = -1;
-        else q = (int8_t)r;                         /* -1, 0 (also -0) or 1 */
+        if (r >= 1.0f) q = 1;
+        else if (r <= -1.0f) q = -1;
+        else q = 0;
         Wq[i] = q;
     }
 }

@@ -94,62 +94,174 @@ __device__ __forceinline__ int quant_code(float t, float inv) {
   return v >= 127.0f ? 127 : (v <= -128.0f ? -128 : static_cast<int>(v));
 }
 
-// Quantise one row (K elements, K % 16 == 0) with the whole CTA (NT
-// threads).  dst receives K int8 codes (generic pointer: shared or global).
-// Returns scale and code sum to every thread.
-template <int NT>
-__device__ void quant_row(const void* row, int x_dtype, int K, const float* __restrict__ gain, float rms_eps,
-                          int8_t* dst, RowRed<NT>& red, float& scale_out, int& sum_out) {
-  float amax = 0.0f;
-  double ss = 0.0;
-  for (int k = threadIdx.x * 8; k < K; k += NT * 8) {
-    float v[8];
-    load8(row, x_dtype, k, v);
-    if (gain != nullptr) {
-      float g[8];
-      load8_gain(gain, k, g);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        amax = fmaxf(amax, fabsf(__fmul_rn(v[i], g[i])));
-        ss = __dadd_rn(ss, __dmul_rn(static_cast<double>(v[i]), static_cast<double>(v[i])));
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(v[i]));
-    }
-  }
-  amax = block_max<NT>(amax, red);
-  if (gain != nullptr) ss = block_sum_d<NT>(ss, red);
-  const float a = fmaxf(amax, kActFloor);
-  const float inv = __fdiv_rn(127.0f, a);
+// Scratch for quant_rows: per-warp partials of up to MT rows.
+template <int NT, int MT>
+struct QuantScratch {
+  float amax[MT][NT / 32];
+  double ss[MT][NT / 32];
+  int qpart[MT][NT / 32];
+};
 
-  int qsum = 0;
-  for (int k = threadIdx.x * 8; k < K; k += NT * 8) {
-    float v[8];
-    load8(row, x_dtype, k, v);
-    if (gain != nullptr) {
-      float g[8];
-      load8_gain(gain, k, g);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], g[i]);
-    }
-    uint32_t lo = 0, hi = 0;
+__device__ __forceinline__ void decode8(const uint4 (&raw)[2], int x_dtype, float (&v)[8]) {
+  if (x_dtype == BITNET_BF16) {
+    const uint32_t w[4] = {raw[0].x, raw[0].y, raw[0].z, raw[0].w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int q0 = quant_code(v[i], inv), q1 = quant_code(v[i + 4], inv);
-      qsum += q0 + q1;
-      lo |= (static_cast<uint32_t>(q0) & 0xffu) << (8 * i);
-      hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);
+      v[2 * i] = bf16_bits_to_float(w[i] & 0xffffu);
+      v[2 * i + 1] = bf16_bits_to_float(w[i] >> 16);
     }
-    *reinterpret_cast<uint2*>(dst + k) = make_uint2(lo, hi);
-  }
-  sum_out = block_sum_i<NT>(qsum, red);
-  if (gain != nullptr) {
-    const double r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, static_cast<double>(K)),
-                                                          static_cast<double>(rms_eps))));
-    scale_out = __double2float_rn(__ddiv_rn(__dmul_rn(r, static_cast<double>(a)), 127.0));
   } else {
-    scale_out = __fdiv_rn(a, 127.0f);
+    v[0] = __uint_as_float(raw[0].x); v[1] = __uint_as_float(raw[0].y);
+    v[2] = __uint_as_float(raw[0].z); v[3] = __uint_as_float(raw[0].w);
+    v[4] = __uint_as_float(raw[1].x); v[5] = __uint_as_float(raw[1].y);
+    v[6] = __uint_as_float(raw[1].z); v[7] = __uint_as_float(raw[1].w);
+  }
+}
+
+__device__ __forceinline__ void load8raw(const char* row, int x_dtype, int k, uint4 (&raw)[2]) {
+  if (x_dtype == BITNET_BF16) {
+    raw[0] = __ldg(reinterpret_cast<const uint4*>(row + 2 * static_cast<int64_t>(k)));
+  } else {
+    const uint4* q = reinterpret_cast<const uint4*>(row + 4 * static_cast<int64_t>(k));
+    raw[0] = __ldg(q);
+    raw[1] = __ldg(q + 1);
+  }
+}
+
+// Quantise rows 0..M-1 (M <= MT, K % 16 == 0) of x with one CTA of NT
+// threads.  Pass 1 finds max|t| (and sum x^2 with a gain) per row, keeping
+// up to C 8-element bfloat16 chunks per thread in registers; one
+// __syncthreads combines the per-warp partials in a fixed order.  Pass 2
+// writes the codes to dst (row stride dst_stride, generic address) and
+// leaves per-warp partial code sums in S.qpart: the caller's next
+// __syncthreads publishes both.  scale[m] is returned to every thread.
+template <int NT, int MT, int C>
+__device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dtype, int64_t row_bytes, int M,
+                                           int K, const float* __restrict__ gain, float rms_eps, int8_t* dst,
+                                           int64_t dst_stride, QuantScratch<NT, MT>& S, float (&scale)[MT]) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const bool cache_ok = (x_dtype == BITNET_BF16);
+  uint4 cache[MT][C];
+  float am[MT];
+  double ss[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    am[m] = 0.0f;
+    ss[m] = 0.0;
+    if (m < M) {
+      const char* row = x + m * row_bytes;
+      auto process = [&](const float (&v)[8], int k) {
+        if (gain != nullptr) {
+          float g[8];
+          load8_gain(gain, k, g);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            am[m] = fmaxf(am[m], fabsf(__fmul_rn(v[i], g[i])));
+            ss[m] = __dadd_rn(ss[m], __dmul_rn(static_cast<double>(v[i]), static_cast<double>(v[i])));
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) am[m] = fmaxf(am[m], fabsf(v[i]));
+        }
+      };
+#pragma unroll
+      for (int c = 0; c < C; ++c) {
+        const int k = (c * NT + tid) * 8;
+        if (k < K) {
+          uint4 raw[2];
+          load8raw(row, x_dtype, k, raw);
+          if (cache_ok) cache[m][c] = raw[0];
+          float v[8];
+          decode8(raw, x_dtype, v);
+          process(v, k);
+        }
+      }
+      for (int k = (C * NT + tid) * 8; k < K; k += NT * 8) {
+        uint4 raw[2];
+        load8raw(row, x_dtype, k, raw);
+        float v[8];
+        decode8(raw, x_dtype, v);
+        process(v, k);
+      }
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    am[m] = warp_max(am[m]);
+    if (gain != nullptr) ss[m] = warp_sum(ss[m]);
+    if (lane == 0) {
+      S.amax[m][warp] = am[m];
+      S.ss[m][warp] = ss[m];
+    }
+  }
+  __syncthreads();
+  float inv[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    float A = S.amax[m][0];
+    double SS = S.ss[m][0];
+#pragma unroll
+    for (int w = 1; w < NT / 32; ++w) {
+      A = fmaxf(A, S.amax[m][w]);
+      SS = __dadd_rn(SS, S.ss[m][w]);
+    }
+    const float a = fmaxf(A, kActFloor);
+    inv[m] = __fdiv_rn(127.0f, a);
+    if (gain != nullptr) {
+      const double r = __ddiv_rn(1.0, __dsqrt_rn(__dadd_rn(__ddiv_rn(SS, static_cast<double>(K)),
+                                                            static_cast<double>(rms_eps))));
+      scale[m] = __double2float_rn(__ddiv_rn(__dmul_rn(r, static_cast<double>(a)), 127.0));
+    } else {
+      scale[m] = __fdiv_rn(a, 127.0f);
+    }
+  }
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    int qs = 0;
+    if (m < M) {
+      const char* row = x + m * row_bytes;
+      int8_t* drow = dst + m * dst_stride;
+      auto emit = [&](float (&v)[8], int k) {
+        if (gain != nullptr) {
+          float g[8];
+          load8_gain(gain, k, g);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], g[i]);
+        }
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int q0 = quant_code(v[i], inv[m]), q1 = quant_code(v[i + 4], inv[m]);
+          qs += q0 + q1;
+          lo |= (static_cast<uint32_t>(q0) & 0xffu) << (8 * i);
+          hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);
+        }
+        *reinterpret_cast<uint2*>(drow + k) = make_uint2(lo, hi);
+      };
+#pragma unroll
+      for (int c = 0; c < C; ++c) {
+        const int k = (c * NT + tid) * 8;
+        if (k < K) {
+          uint4 raw[2];
+          if (cache_ok)
+            raw[0] = cache[m][c];
+          else
+            load8raw(row, x_dtype, k, raw);
+          float v[8];
+          decode8(raw, x_dtype, v);
+          emit(v, k);
+        }
+      }
+      for (int k = (C * NT + tid) * 8; k < K; k += NT * 8) {
+        uint4 raw[2];
+        load8raw(row, x_dtype, k, raw);
+        float v[8];
+        decode8(raw, x_dtype, v);
+        emit(v, k);
+      }
+    }
+    qs = warp_sum(qs);
+    if (lane == 0) S.qpart[m][warp] = qs;
   }
 }
 
@@ -160,19 +272,22 @@ __global__ void __launch_bounds__(kActThreads) quant_act_kernel(const void* __re
                                                                 const float* __restrict__ gain, float rms_eps,
                                                                 int8_t* __restrict__ xq, float* __restrict__ x_scale,
                                                                 int32_t* __restrict__ x_sum) {
-  __shared__ RowRed<kActThreads> red;
+  __shared__ QuantScratch<kActThreads, 1> S;
+  pdl_launch_dependents();
   pdl_wait();
   const int64_t m = blockIdx.x;
-  const size_t esz = (x_dtype == BITNET_BF16) ? 2 : 4;
-  const void* row = static_cast<const char*>(x) + m * K * esz;
-  float s;
-  int qs;
-  quant_row<kActThreads>(row, x_dtype, K, gain, rms_eps, xq + m * K, red, s, qs);
+  const int64_t esz = (x_dtype == BITNET_BF16) ? 2 : 4;
+  float sc[1];
+  quant_rows<kActThreads, 1, 2>(static_cast<const char*>(x) + m * K * esz, x_dtype, K * esz, 1, K, gain, rms_eps,
+                                xq + m * K, K, S, sc);
+  __syncthreads();
   if (threadIdx.x == 0) {
-    x_scale[m] = s;
-    if (x_sum != nullptr) x_sum[m] = qs;
+    int t = 0;
+#pragma unroll
+    for (int w = 0; w < kActThreads / 32; ++w) t += S.qpart[0][w];
+    x_scale[m] = sc[0];
+    if (x_sum != nullptr) x_sum[m] = t;
   }
-  pdl_launch_dependents();
 }
 
 // Row sums of pre-quantised activations (when a caller gives no x_sum).

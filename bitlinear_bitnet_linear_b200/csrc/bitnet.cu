@@ -100,9 +100,34 @@ cudaError_t launch_pdl(Kern kernel, dim3 grid, dim3 block, size_t smem, cudaStre
   return cudaLaunchKernelEx(&cfg, kernel, args...);
 }
 
+// Raise a kernel's dynamic shared-memory limit once per (kernel, device):
+// the attribute call is host work that must not recur on every launch (and
+// must not be needed inside a stream capture once warmed up).
 template <typename Kern>
 cudaError_t allow_smem(Kern kernel, size_t bytes) {
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  struct Entry {
+    const void* fn;
+    int dev;
+    size_t bytes;
+  };
+  static Entry cache[256];
+  static int used = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaErrorInvalidDevice;
+  const void* fn = reinterpret_cast<const void*>(kernel);
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].fn == fn && cache[i].dev == dev) {
+      if (cache[i].bytes >= bytes) return cudaSuccess;
+      cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           static_cast<int>(bytes));
+      if (e == cudaSuccess) cache[i].bytes = bytes;
+      return e;
+    }
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e == cudaSuccess && used < 256) cache[used++] = Entry{fn, dev, bytes};
+  return e;
 }
 
 int elementwise_grid(int64_t work, const DeviceInfo* d) {
@@ -144,32 +169,37 @@ struct GemvPlan {
 
 bitnet_status plan_gemv(const DeviceInfo* d, int64_t M, int64_t K, int64_t N, GemvPlan& pl) {
   if (M > kGemvMaxM) return BITNET_ERR_UNSUPPORTED;
-  pl.MT = M <= 1 ? 1 : (M <= 2 ? 2 : 4);
-  pl.R = K <= 4096 ? 4 : (K <= 8192 ? 2 : 1);
-  if (pl.MT == 4 && pl.R == 4) pl.R = 2;
   GemvParams& p = pl.p;
+  pl.MT = M <= 1 ? 1 : (M <= 2 ? 2 : 4);
   p.M = static_cast<int>(M);
   p.K = static_cast<int>(K);
   p.N = static_cast<int>(N);
   p.Kp = static_cast<int>(round_up(static_cast<size_t>(K), 64));
   p.bulk = (K % 64 == 0) ? 1 : 0;
   p.wrow = p.bulk ? static_cast<int>(K / 4) : p.Kp / 4;
-  const int grid = static_cast<int>(N < d->sms ? N : d->sms);
+  // Two CTAs per SM: each is latency-bound on its own, two overlap.
+  const int64_t cap = 2 * static_cast<int64_t>(d->sms);
+  const int grid = static_cast<int>(N < cap ? N : cap);
   pl.grid = grid;
   p.rows_base = static_cast<int>(N / grid);
   p.rows_extra = static_cast<int>(N % grid);
   const int rows_cta = p.rows_base + (p.rows_extra ? 1 : 0);
+  // rows per warp task: enough tasks for all eight warps, more ILP when rows abound
+  if (rows_cta <= kGvWarps) pl.R = 1;
+  else if (rows_cta <= 2 * kGvWarps) pl.R = 2;
+  else pl.R = K <= 4096 ? 4 : (K <= 8192 ? 2 : 1);
+  if (pl.MT == 4 && pl.R == 4) pl.R = 2;
   const int xbytes = pl.MT * p.Kp;
   // Prefer a footprint that lets the next call's CTAs co-reside (PDL
-  // overlap); grow only when one stage would not fit.
-  const int budget_soft = 112 * 1024;
+  // overlap); grow only when two stages would not fit.
+  const int budget_soft = 96 * 1024;
   const int budget_hard = d->max_smem_optin;
   int stage_rows = kGvWarps * pl.R;
   if (stage_rows > rows_cta) stage_rows = rows_cta;
   const int stage_bytes = stage_rows * p.wrow;
   const int nst = (rows_cta + stage_rows - 1) / stage_rows;
   int room = budget_soft - kGvHeader - xbytes;
-  if (room < 2 * stage_bytes) room = budget_hard - kGvHeader - xbytes;
+  if (room < 2 * stage_bytes && nst > 1) room = budget_hard - kGvHeader - xbytes;
   int stages = room / stage_bytes;
   if (stages > kGvMaxStages) stages = kGvMaxStages;
   if (stages > nst) stages = nst;
@@ -207,7 +237,7 @@ cudaError_t run_gemv(const GemvPlan& pl, cudaStream_t st) {
 // ---------------------------------------------------------------------------
 // Tensor-core GEMM launch.
 // ---------------------------------------------------------------------------
-template <int BM, int STAGES>
+template <int BM, int SS, int AS>
 cudaError_t run_tc_t(const int8_t* xq, const TcParams& p, cudaStream_t st) {
   CUtensorMap map;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.K), static_cast<cuuint64_t>(p.M)};
@@ -218,20 +248,21 @@ cudaError_t run_tc_t(const int8_t* xq, const TcParams& p, cudaStream_t st) {
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto k = tc_gemm_kernel<BM, STAGES>;
-  constexpr int smem = tc_smem_bytes<BM, STAGES>();
+  auto k = tc_gemm_kernel<BM, SS, AS>;
+  constexpr int smem = tc_smem_bytes<BM, SS>();
   cudaError_t e = allow_smem(k, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((p.N + kTcBN - 1) / kTcBN, (p.M + BM - 1) / BM);
   return launch_pdl(k, grid, dim3(kTcThreads), smem, st, map, p);
 }
 
+// Token tile BM = MMA N.  With 4 TMEM A buffers every configuration holds at
+// most 256 TMEM columns, so two CTAs can share an SM.
 cudaError_t run_tc(const int8_t* xq, const TcParams& p, cudaStream_t st) {
-  if (p.M <= 16) return run_tc_t<16, 8>(xq, p, st);
-  if (p.M <= 32) return run_tc_t<32, 8>(xq, p, st);
-  if (p.M <= 64) return run_tc_t<64, 8>(xq, p, st);
-  if (p.M <= 128) return run_tc_t<128, 6>(xq, p, st);
-  return run_tc_t<256, 4>(xq, p, st);
+  if (p.M <= 16) return run_tc_t<16, 8, 4>(xq, p, st);
+  if (p.M <= 32) return run_tc_t<32, 8, 4>(xq, p, st);
+  if (p.M <= 64) return run_tc_t<64, 8, 4>(xq, p, st);
+  return run_tc_t<128, 6, 4>(xq, p, st);
 }
 
 bitnet_status launch_result(cudaError_t e) {

@@ -17,10 +17,13 @@
 //   warp 0       TMA producer: activation tiles [BM x 128 B], 128-byte swizzle
 //   warp 1       TMEM allocator and single-thread MMA issuer
 //   warps 2..5   converters (one weight row per thread), then the epilogue
-// Pipeline: STAGES slots; slot s has an activation buffer in shared memory and
-// a 32-column A buffer in TMEM.  mbarriers: full[s] (TMA bytes landed),
-// afull[s] (128 converter threads stored codes), empty[s] (the MMAs that read
-// slot s completed; tcgen05.commit), accf (all MMAs completed).
+// Pipeline: SS activation stages in shared memory and AS 32-column A buffers
+// in TMEM, cycled independently.  mbarriers: full[s] (TMA bytes landed),
+// sempty[s] (MMAs that read stage s completed; tcgen05.commit), afull[a] (128
+// converter threads stored codes), aempty[a] (MMAs that read A buffer a
+// completed), accf (all MMAs completed).  With BM <= 128 and AS = 4 a CTA
+// holds 256 TMEM columns, so two CTAs share an SM and one's epilogue
+// overlaps the other's main loop.
 // Every wait is bounded; on expiry the kernel records BITNET_ERR_TIMEOUT,
 // raises a CTA-wide abort flag, drains what it issued and frees TMEM.
 #pragma once
@@ -48,14 +51,14 @@ struct TcParams {
   uint32_t* status;
 };
 
-__host__ __device__ constexpr uint32_t tc_tmem_cols(int BM, int STAGES) {
-  const int need = BM + 32 * STAGES;
+__host__ __device__ constexpr uint32_t tc_tmem_cols(int BM, int AS) {
+  const int need = BM + 32 * AS;
   return need <= 32 ? 32u : need <= 64 ? 64u : need <= 128 ? 128u : need <= 256 ? 256u : 512u;
 }
 
-template <int BM, int STAGES>
+template <int BM, int SS>
 __host__ __device__ constexpr int tc_smem_bytes() {
-  return 1024 /* alignment slack */ + STAGES * BM * kTcBK + 256 /* barriers, flags */;
+  return 1024 /* alignment slack */ + SS * BM * kTcBK + 512 /* barriers, flags */;
 }
 
 // Read the packed codes of one weight row for K block kb (32 bytes = 128
@@ -83,12 +86,12 @@ __device__ __forceinline__ void tc_load_row_block(const uint8_t* __restrict__ ro
   }
 }
 
-template <int BM, int STAGES>
+template <int BM, int SS, int AS>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
   static_assert(BM % 16 == 0 && BM >= 16 && BM <= 256, "MMA N must be a multiple of 16 in [16, 256]");
-  constexpr uint32_t kCols = tc_tmem_cols(BM, STAGES);
-  constexpr uint32_t kACol0 = BM;                  // A buffer s at columns [BM + 32 s, BM + 32 s + 32)
+  constexpr uint32_t kCols = tc_tmem_cols(BM, AS);
+  constexpr uint32_t kACol0 = BM;                  // A buffer a at columns [BM + 32 a, BM + 32 a + 32)
   constexpr uint32_t kStageBytes = BM * kTcBK;
   constexpr uint32_t kIdesc = idesc_i8_us(kTcBN, BM);
   constexpr int kPD = 4;                           // converter prefetch depth (K blocks)
@@ -96,10 +99,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * kStageBytes);
-  uint64_t* empty = full + STAGES;
-  uint64_t* afull = empty + STAGES;
-  uint64_t* accf = afull + STAGES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SS * kStageBytes);
+  uint64_t* sempty = full + SS;
+  uint64_t* afull = sempty + SS;
+  uint64_t* aempty = afull + AS;
+  uint64_t* accf = aempty + AS;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(accf + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -109,10 +113,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int KB = p.KB;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < SS; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-      mbar_init(&afull[s], 128);
+      mbar_init(&sempty[s], 1);
+    }
+    for (int a = 0; a < AS; ++a) {
+      mbar_init(&afull[a], 128);
+      mbar_init(&aempty[a], 1);
     }
     mbar_init(accf, 1);
     *abort_flag = 0;
@@ -139,9 +146,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       pdl_wait();   // activations come from the previous kernel
       int issued = 0;
       for (int kb = 0; kb < KB; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        if (!mbar_wait_bounded(&empty[s], ph ^ 1u, p.limit_ns, abort_flag)) {
+        const int s = kb % SS;
+        const uint32_t ph = (kb / SS) & 1;
+        if (!mbar_wait_bounded(&sempty[s], ph ^ 1u, p.limit_ns, abort_flag)) {
           if (!*abort_flag) fail(0x301u);
           break;
         }
@@ -151,8 +158,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (*abort_flag) {
         // drain: let every copy already issued land before the CTA can exit
-        for (int kb = max(0, issued - STAGES); kb < issued; ++kb)
-          mbar_wait_bounded(&full[kb % STAGES], (kb / STAGES) & 1, p.limit_ns, nullptr);
+        for (int kb = max(0, issued - SS); kb < issued; ++kb)
+          mbar_wait_bounded(&full[kb % SS], (kb / SS) & 1, p.limit_ns, nullptr);
       }
     }
   } else if (warp == 1) {
@@ -160,10 +167,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       bool ok = true;
       for (int kb = 0; kb < KB && ok; ++kb) {
-        const int s = kb % STAGES;
-        const uint32_t ph = (kb / STAGES) & 1;
-        if (!mbar_wait_bounded(&full[s], ph, p.limit_ns, abort_flag) ||
-            !mbar_wait_bounded(&afull[s], ph, p.limit_ns, abort_flag)) {
+        const int s = kb % SS;
+        const int a = kb % AS;
+        if (!mbar_wait_bounded(&full[s], (kb / SS) & 1, p.limit_ns, abort_flag) ||
+            !mbar_wait_bounded(&afull[a], (kb / AS) & 1, p.limit_ns, abort_flag)) {
           if (!*abort_flag) fail(0x302u);
           ok = false;
           break;
@@ -173,10 +180,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int j = 0; j < kTcBK / 32; ++j) {
           // K step of 32 bytes: advance the descriptor start address by 32 B (>> 4 = 2)
-          tc_mma_i8_ts(tmem, tmem + kACol0 + 32u * s + 8u * j, bdesc + 2ull * j, kIdesc,
+          tc_mma_i8_ts(tmem, tmem + kACol0 + 32u * a + 8u * j, bdesc + 2ull * j, kIdesc,
                        (kb | j) != 0 ? 1u : 0u);
         }
-        tc_commit(&empty[s]);
+        tc_commit(&sempty[s]);
+        tc_commit(&aempty[a]);
       }
       // Completion of everything issued so far (also on abort: nothing may
       // still read TMEM when it is freed).
@@ -204,9 +212,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int j = 0; j < kPD; ++j) {
         const int kb = kb0 + j;
         if (kb < KB && ok) {
-          const int s = kb % STAGES;
-          const uint32_t ph = (kb / STAGES) & 1;
-          if (!mbar_wait_bounded(&empty[s], ph ^ 1u, p.limit_ns, abort_flag)) {
+          const int a = kb % AS;
+          const uint32_t ph = (kb / AS) & 1;
+          if (!mbar_wait_bounded(&aempty[a], ph ^ 1u, p.limit_ns, abort_flag)) {
             if (!*abort_flag) fail(0x303u);
             ok = false;
           }
@@ -222,10 +230,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               codes[4 * g + 2] = (w >> 4) & 0x03030303u;
               codes[4 * g + 3] = (w >> 6) & 0x03030303u;
             }
-            tmem_st_32x32b_x32(tmem + lane_base + kACol0 + 32u * s, codes);
+            tmem_st_32x32b_x32(tmem + lane_base + kACol0 + 32u * a, codes);
             tc_wait_st();
             tc_fence_before();
-            mbar_arrive(&afull[s]);
+            mbar_arrive(&afull[a]);
             if (kb + kPD < KB) tc_load_row_block(wrow, valid, rowbytes, kb + kPD, p.wvec, wb[j]);
           } else {
             ok = false;
@@ -240,23 +248,32 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       pdl_wait();   // token scales and sums come from the previous kernel
       pdl_launch_dependents();
       const float gamma = __ldg(p.gamma);
+      const float* __restrict__ xsc = p.x_scale;
+      const int32_t* __restrict__ xsm = p.x_sum;
 #pragma unroll 1
       for (int c0 = 0; c0 < BM; c0 += 32) {
         if (m0 + c0 >= p.M) break;   // warp-uniform
+        // lane i fetches token (m0 + c0 + i)'s constants once; shuffled below
+        const int mi = m0 + c0 + lane;
+        float gs = 0.0f;
+        int xsum = 0;
+        if (mi < p.M) {
+          gs = __fmul_rn(gamma, __ldg(xsc + mi));
+          xsum = __ldg(xsm + mi);
+        }
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem + lane_base + static_cast<uint32_t>(c0), v);
         tc_wait_ld();
-        if (valid) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const int m = m0 + c0 + i;
-            if (m < p.M) {
-              const int a = static_cast<int>(v[i]) - __ldg(p.x_sum + m);
-              const int64_t idx = static_cast<int64_t>(m) * p.N + n;
-              if (p.acc != nullptr) p.acc[idx] = a;
-              if (p.y != nullptr)
-                store_y(p.y, p.y_dtype, idx, __fmul_rn(__int2float_rn(a), __fmul_rn(gamma, __ldg(p.x_scale + m))));
-            }
+        for (int i = 0; i < 32; ++i) {
+          const float gsi = __shfl_sync(0xffffffffu, gs, i);
+          const int xsi = __shfl_sync(0xffffffffu, xsum, i);
+          const int m = m0 + c0 + i;
+          if (valid && m < p.M) {
+            const int a = static_cast<int>(v[i]) - xsi;
+            const int64_t idx = static_cast<int64_t>(m) * p.N + n;
+            if (p.acc != nullptr) p.acc[idx] = a;
+            if (p.y != nullptr) store_y(p.y, p.y_dtype, idx, __fmul_rn(__int2float_rn(a), gsi));
           }
         }
       }

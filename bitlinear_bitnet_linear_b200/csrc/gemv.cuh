@@ -31,7 +31,7 @@ namespace bitnet {
 constexpr int kGvThreads = 256;
 constexpr int kGvWarps = kGvThreads / 32;
 constexpr int kGvMaxStages = 8;
-constexpr int kGvHeader = 1024;   // barriers + reduction scratch + per-token scale/sum
+constexpr int kGvHeader = 1024;   // barriers + reduction scratch + per-token scale
 
 struct GemvParams {
   // activations: either raw x (fused quantiser) or pre-quantised x_q
@@ -62,9 +62,8 @@ struct GemvParams {
 template <int MT>
 struct GemvHeader {
   uint64_t full[kGvMaxStages];
-  RowRed<kGvThreads> red;
+  QuantScratch<kGvThreads, MT> q;
   float scale[MT];
-  int sum[MT];
 };
 
 template <int MT, int R, bool FUSED>
@@ -92,62 +91,56 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(const GemvParams p) {
     bulk_g2s(ring + s * stage_bytes, p.Wp + (n0 + r0) * rowbytes, bytes, &H.full[s]);
   };
 
-  if (tid == 0) {
+  // Weights never depend on earlier kernels: start streaming them at once.
+  // The first __syncthreads below orders this initialisation before any
+  // other thread waits on the barriers.
+  if (tid == 0 && p.bulk) {
     for (int s = 0; s < p.stages; ++s) mbar_init(&H.full[s], 1);
     fence_mbar_init();
-  }
-  __syncthreads();
-  if (p.bulk && tid == 0) {
     for (int i = 0; i < min(p.stages, nst); ++i) issue(i);
   }
-
-  // Everything above touched only the (read-only) weights.
+  // Let the next kernel in the stream launch and start its own weight
+  // stream; it still waits for this grid before touching our outputs.
+  pdl_launch_dependents();
   pdl_wait();
 
   // ---- prologue: activation codes into shared memory, zero padded --------
-  for (int m = 0; m < MT; ++m) {
-    int8_t* xrow = xs + m * p.Kp;
-    if (m < p.M) {
-      if constexpr (FUSED) {
-        const size_t esz = (p.x_dtype == BITNET_BF16) ? 2 : 4;
-        float s;
-        int qs;
-        quant_row<kGvThreads>(static_cast<const char*>(p.x) + static_cast<int64_t>(m) * p.K * esz, p.x_dtype,
-                              p.K, p.gain, p.rms_eps, xrow, H.red, s, qs);
-        if (tid == 0) {
-          H.scale[m] = s;
-          H.sum[m] = qs;
-        }
-      } else {
-        int part = 0;
+  if constexpr (FUSED) {
+    const int64_t esz = (p.x_dtype == BITNET_BF16) ? 2 : 4;
+    float sc[MT];
+    quant_rows<kGvThreads, MT, (MT == 1 ? 4 : (MT == 2 ? 2 : 1))>(static_cast<const char*>(p.x), p.x_dtype,
+                                                                 p.K * esz, p.M, p.K, p.gain, p.rms_eps, xs, p.Kp,
+                                                                 H.q, sc);
+    if (tid == 0) {
+#pragma unroll
+      for (int m = 0; m < MT; ++m) H.scale[m] = sc[m];
+    }
+  } else {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      int part = 0;
+      if (m < p.M) {
         for (int k = tid * 16; k < p.K; k += kGvThreads * 16) {
           const uint4 u = __ldg(reinterpret_cast<const uint4*>(p.xq + static_cast<int64_t>(m) * p.K + k));
-          *reinterpret_cast<uint4*>(xrow + k) = u;
+          *reinterpret_cast<uint4*>(xs + m * p.Kp + k) = u;
           part = __dp4a(static_cast<int>(u.x), 0x01010101, part);
           part = __dp4a(static_cast<int>(u.y), 0x01010101, part);
           part = __dp4a(static_cast<int>(u.z), 0x01010101, part);
           part = __dp4a(static_cast<int>(u.w), 0x01010101, part);
         }
-        const int qs = block_sum_i<kGvThreads>(part, H.red);
-        if (tid == 0) {
-          H.scale[m] = __ldg(p.x_scale + m);
-          H.sum[m] = qs;
-        }
       }
-      for (int k = p.K + tid * 16; k < p.Kp; k += kGvThreads * 16)
-        *reinterpret_cast<uint4*>(xrow + k) = make_uint4(0, 0, 0, 0);
-    } else {
-      for (int k = tid * 16; k < p.Kp; k += kGvThreads * 16)
-        *reinterpret_cast<uint4*>(xrow + k) = make_uint4(0, 0, 0, 0);
-      if (tid == 0) {
-        H.scale[m] = 0.0f;
-        H.sum[m] = 0;
-      }
+      part = warp_sum(part);
+      if (lane == 0) H.q.qpart[m][warp] = part;
+      if (tid == 0) H.scale[m] = (m < p.M) ? __ldg(p.x_scale + m) : 0.0f;
     }
   }
+  for (int m = 0; m < MT; ++m) {
+    const int k0 = (m < p.M) ? p.K : 0;
+    for (int k = k0 + tid * 16; k < p.Kp; k += kGvThreads * 16)
+      *reinterpret_cast<uint4*>(xs + m * p.Kp + k) = make_uint4(0, 0, 0, 0);
+    if (m >= p.M && lane == 0) H.q.qpart[m][warp] = 0;
+  }
   __syncthreads();
-  // The next kernel in the stream may start its own weight prefetch now.
-  pdl_launch_dependents();
 
   const float gamma = __ldg(p.gamma);
   const int nchunk = p.Kp / 64;   // 16-byte chunks (64 weights) per row
@@ -229,7 +222,10 @@ __global__ void __launch_bounds__(kGvThreads) gemv_kernel(const GemvParams p) {
         for (int m = 0; m < MT; ++m) {
           if (lane == r * MT + m && r < nr && m < p.M) {
             const int64_t n = n0 + r0 + rg * R + r;
-            const int accv = a[r][m][0] - H.sum[m];
+            int xsum = 0;
+#pragma unroll
+            for (int w = 0; w < kGvWarps; ++w) xsum += H.q.qpart[m][w];
+            const int accv = a[r][m][0] - xsum;
             const int64_t idx = static_cast<int64_t>(m) * p.N + n;
             if (p.acc != nullptr) p.acc[idx] = accv;
             if (p.y != nullptr) store_y(p.y, p.y_dtype, idx, __fmul_rn(__int2float_rn(accv), __fmul_rn(gamma, H.scale[m])));

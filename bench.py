@@ -51,6 +51,7 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-chain", action="store_true")
     ap.add_argument("--prefill-iters", type=int, default=50)
     ap.add_argument("--only", choices=["all", "decode", "prefill"], default="all",
                     help="run one part (for profiling a single kernel on a small case)")
@@ -177,50 +178,76 @@ def run_ours(args):
 
     bytes_step = sum(N * K // 4 + K * 2 + N * 2 + 4 for (K, N, _, _) in stack)
     calls = len(stack)
+    problems = [(x, Wp, g, gains[K], y) for (K, N, Wp, g), x, y in zip(stack, xs, ys)]
+    grouped = bn.GroupedCall(problems, rms_eps=1e-5, ws=ws)
 
     def step():
+        grouped()
+
+    def chain_step():
         for (K, N, Wp, g), x, y in zip(stack, xs, ys):
             bn.bitnet_linear(x, Wp, g, N=N, rms_gain=gains[K], rms_eps=1e-5, y=y, ws=ws)
-
-    # warm up eagerly, then capture one step in a CUDA graph (PDL edges kept)
-    with torch.cuda.stream(stream):
-        for _ in range(2):
-            step()
-    torch.cuda.synchronize()
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        step()
-    torch.cuda.synchronize()
-    assert bn.bitnet_get_error(ws) == 0
 
     def barrier():
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
 
-    for _ in range(max(3, args.warmup)):
-        graph.replay()
-    barrier()
-    clocks = ClockSampler(dev.index)
-    clocks.start()
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    barrier()
-    with torch.cuda.stream(stream):
-        e0.record(stream)
-        for _ in range(args.steps):
-            graph.replay()
-        e1.record(stream)
-    barrier()
-    clk = clocks.stop()
-    ms = e0.elapsed_time(e1) / args.steps
-    t = torch.tensor([ms], device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_max = float(t.item())
+    def capture(fn):
+        with torch.cuda.stream(stream):
+            for _ in range(2):
+                fn()
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            fn()
+        torch.cuda.synchronize()
+        assert bn.bitnet_get_error(ws) == 0
+        return gr
+
+    def time_graph(gr, steps, warm, sample_clocks=False):
+        for _ in range(max(3, warm)):
+            gr.replay()
+        barrier()
+        clk = None
+        sampler = ClockSampler(dev.index) if sample_clocks else None
+        if sampler:
+            sampler.start()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        barrier()
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(steps):
+                gr.replay()
+            e1.record(stream)
+        barrier()
+        if sampler:
+            clk = sampler.stop()
+        ms_local = e0.elapsed_time(e1) / steps
+        t = torch.tensor([ms_local], device=dev)
+        if world > 1:
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return ms_local, float(t.item()), clk
+
+    graph = capture(step)
+    ms, ms_max, clk = time_graph(graph, args.steps, args.warmup, sample_clocks=True)
     assert bn.bitnet_get_error(ws) == 0
     value = world * bytes_step / (ms_max * 1e-3) / 1e9
     per_rank = bytes_step / (ms * 1e-3) / 1e9
+
+    # ---- the same 210 calls as a dependent chain of separate launches ------
+    chain = None
+    if not args.no_chain:
+        cgraph = capture(chain_step)
+        csteps = max(20, args.steps // 10)
+        cms, cms_max, _ = time_graph(cgraph, csteps, 3)
+        chain = {"value": round(world * bytes_step / (cms_max * 1e-3) / 1e9, 2), "unit": "GB/s",
+                 "ms_per_step": round(cms_max, 4), "us_per_call": round(cms_max * 1e3 / calls, 3),
+                 "steps": csteps, "launches_per_step": calls,
+                 "what": "each of the 210 calls its own bitnet_linear launch, in stream order (each waits for "
+                         "the previous), programmatic dependent launch, one CUDA graph per step"}
+        del cgraph
 
     # ---- e2e: host buffers, through the public API, no graph ----------------
     e2e = None
@@ -242,18 +269,20 @@ def run_ours(args):
             o += y.numel()
         xviews = [x_dev[a:a + k].view(1, k) for a, k in xo]
         yviews = [y_dev[a:a + n].view(1, n) for a, n in yo]
+        eproblems = [(x, Wp, g, gains[K], y) for (K, N, Wp, g), x, y in zip(stack, xviews, yviews)]
 
         def e2e_step():
             x_dev.copy_(x_pin, non_blocking=True)
-            for (K, N, Wp, g), x, y in zip(stack, xviews, yviews):
-                bn.bitnet_linear(x, Wp, g, N=N, rms_gain=gains[K], rms_eps=1e-5, y=y, ws=ws)
+            bn.bitnet_linear_grouped(eproblems, rms_eps=1e-5, ws=ws)
             y_pin.copy_(y_dev, non_blocking=True)
 
-        e2e_steps = max(5, min(200, args.steps // 10))
+        e2e_steps = max(10, min(500, args.steps // 4))
         with torch.cuda.stream(stream):
             for _ in range(3):
                 e2e_step()
         barrier()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(stream):
             e0.record(stream)
             for _ in range(e2e_steps):
@@ -266,25 +295,7 @@ def run_ours(args):
             dist.all_reduce(te, op=dist.ReduceOp.MAX)
         e2e = {"value": round(world * bytes_step / (float(te.item()) * 1e-3) / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(float(te.item()), 4),
-               "path": "python binding -> C ABI bitnet_linear per call, no graph"}
-        # same, with the step's 210 calls replayed from the captured graph
-        ge = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(ge, stream=stream):
-            for (K, N, Wp, g), x, y in zip(stack, xviews, yviews):
-                bn.bitnet_linear(x, Wp, g, N=N, rms_gain=gains[K], rms_eps=1e-5, y=y, ws=ws)
-        barrier()
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(e2e_steps):
-                x_dev.copy_(x_pin, non_blocking=True)
-                ge.replay()
-                y_pin.copy_(y_dev, non_blocking=True)
-            e1.record(stream)
-        barrier()
-        gms = e0.elapsed_time(e1) / e2e_steps
-        e2e["graph_value"] = round(bytes_step / (gms * 1e-3) / 1e9, 2)
-        e2e["graph_ms_per_step"] = round(gms, 4)
-        del ge
+               "path": "python binding -> C ABI bitnet_linear_grouped (210 problems), pinned host x in, y out"}
 
     # ---- prefill GEMM (secondary) ------------------------------------------
     prefill = None
@@ -312,20 +323,23 @@ def run_ours(args):
                    "bytes_per_step_per_gpu": bytes_step,
                    "l2": "inputs larger than L2 (594.7 MB of packed weights per step per GPU)",
                    "parallelism": f"dp{world} (independent replicas, no data-path collective)",
-                   "launch": "one CUDA graph per step, programmatic dependent launch between calls"},
+                   "launch": "the step's 210 independent calls as one grouped launch (bitnet_linear_grouped), "
+                             "replayed from a CUDA graph"},
         "tokens_per_s": round(world * 1e3 / ms_max, 1),
-        "roofline": {"bound": "hbm", "kernel": "gemv_kernel<1,4|2,true> (fused quantise + GEMV)",
+        "roofline": {"bound": "hbm", "kernel": "gemv_stream_kernel<1,2,256> (grouped fused quantise + GEMV)",
                      "achieved": round(per_rank, 2), "peak": hbm_peak, "unit": "GB/s",
                      "frac": round(per_rank / hbm_peak, 4), "peak_source": f"{peak_src} HBM copy bandwidth",
                      "frac_of_8TBs_datasheet": round(per_rank / 8000.0, 4),
                      "traffic": None,
-                     "note": "every launch in the timed step is this kernel; achieved = algorithmic bytes "
-                             "per launch / mean launch duration = bytes per step / step time"},
-        "gpu_launches": calls * args.steps,
+                     "note": "one launch of this kernel per step; achieved = algorithmic bytes per launch / "
+                             "mean launch duration"},
+        "gpu_launches": args.steps,
         "clocks": clk,
     }
     if e2e is not None:
         out["e2e"] = e2e
+    if chain is not None:
+        out["decode_chain"] = chain
     if prefill is not None:
         out["prefill"] = prefill
     if cpu is not None:

@@ -26,7 +26,15 @@ PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
 EXPORTS = ("bitnet_workspace_bytes", "bitnet_quant_weights_workspace_bytes", "bitnet_workspace_init",
            "bitnet_get_error", "bitnet_status_str", "bitnet_quant_weights", "bitnet_ternarise",
            "bitnet_pack", "bitnet_unpack", "bitnet_quant_act", "bitnet_linear", "bitnet_linear_ex",
-           "bitnet_linear_q", "bitnet_set_wait_limit_us", "bitnet_watchdog_selftest")
+           "bitnet_linear_q", "bitnet_linear_grouped", "bitnet_set_wait_limit_us",
+           "bitnet_watchdog_selftest")
+
+
+class GemvProblem(ctypes.Structure):
+    """Mirror of bitnet_gemv_problem (include/bitnet.h)."""
+    _fields_ = [("x", ctypes.c_void_p), ("Wp", ctypes.c_void_p), ("gamma", ctypes.c_void_p),
+                ("rms_gain", ctypes.c_void_p), ("y", ctypes.c_void_p), ("K", ctypes.c_int64),
+                ("N", ctypes.c_int64)]
 
 
 class BitnetError(RuntimeError):
@@ -62,6 +70,7 @@ def lib() -> ctypes.CDLL:
         "bitnet_linear": ([P, I32, I64, I64, P, I64, P, P, F, P, I32, P, SZ, P], I32),
         "bitnet_linear_ex": ([P, I32, I64, I64, P, I64, P, P, F, P, I32, P, SZ, I32, P], I32),
         "bitnet_linear_q": ([P, P, P, I64, I64, P, I64, P, P, I32, P, P, SZ, I32, P], I32),
+        "bitnet_linear_grouped": ([P, I32, I64, I32, F, I32, P, SZ, P], I32),
         "bitnet_set_wait_limit_us": ([U32], I32),
         "bitnet_watchdog_selftest": ([P, SZ, U32, P], I32),
     }
@@ -243,3 +252,46 @@ def bitnet_linear_q(xq: torch.Tensor, x_scale: torch.Tensor, Wp: torch.Tensor, g
                                  _ptr(acc) if want_acc else None, _ptr(ws), ws.numel(), int(path),
                                  _stream(stream)), "bitnet_linear_q")
     return y, acc
+
+
+def bitnet_linear_grouped(problems, rms_eps: float = 1e-5, ws=None, stream=None, _keep=None):
+    """problems: sequence of (x, Wp, gamma, rms_gain or None, y) device tensors,
+    all with the same M rows and dtypes.  One launch; see include/bitnet.h."""
+    arr = (GemvProblem * len(problems))()
+    M = problems[0][0].shape[0]
+    xd = _xdtype(problems[0][0])
+    yd = _ydtype(problems[0][4].dtype)
+    for i, (x, Wp, gamma, gain, y) in enumerate(problems):
+        if x.shape[0] != M or _xdtype(x) != xd or _ydtype(y.dtype) != yd:
+            raise ValueError("all problems need the same M and dtypes")
+        arr[i] = GemvProblem(_ptr(x).value, _ptr(Wp).value, _ptr(gamma).value,
+                             None if gain is None else _ptr(gain).value, _ptr(y).value,
+                             x.shape[1], Wp.shape[0])
+    if ws is None:
+        ws = new_workspace(256, problems[0][0].device)
+    _check(lib().bitnet_linear_grouped(ctypes.cast(arr, ctypes.c_void_p), len(problems), M, xd, float(rms_eps), yd,
+                                       _ptr(ws), ws.numel(), _stream(stream)), "bitnet_linear_grouped")
+
+
+class GroupedCall:
+    """A prepared grouped call: the problem table is built once and reused
+    (for CUDA-graph capture or repeated launches)."""
+
+    def __init__(self, problems, rms_eps: float = 1e-5, ws=None):
+        self.arr = (GemvProblem * len(problems))()
+        self.M = problems[0][0].shape[0]
+        self.xd = _xdtype(problems[0][0])
+        self.yd = _ydtype(problems[0][4].dtype)
+        self.keep = list(problems)
+        for i, (x, Wp, gamma, gain, y) in enumerate(problems):
+            self.arr[i] = GemvProblem(_ptr(x).value, _ptr(Wp).value, _ptr(gamma).value,
+                                      None if gain is None else _ptr(gain).value, _ptr(y).value,
+                                      x.shape[1], Wp.shape[0])
+        self.n = len(problems)
+        self.eps = float(rms_eps)
+        self.ws = ws if ws is not None else new_workspace(256, problems[0][0].device)
+
+    def __call__(self, stream=None):
+        _check(lib().bitnet_linear_grouped(ctypes.cast(self.arr, ctypes.c_void_p), self.n, self.M, self.xd,
+                                           self.eps, self.yd, _ptr(self.ws), self.ws.numel(), _stream(stream)),
+               "bitnet_linear_grouped")

@@ -118,14 +118,34 @@ __device__ __forceinline__ void decode8(const uint4 (&raw)[2], int x_dtype, floa
   }
 }
 
+template <bool SMEM_SRC = false>
 __device__ __forceinline__ void load8raw(const char* row, int x_dtype, int k, uint4 (&raw)[2]) {
   if (x_dtype == BITNET_BF16) {
-    raw[0] = __ldg(reinterpret_cast<const uint4*>(row + 2 * static_cast<int64_t>(k)));
+    const uint4* q = reinterpret_cast<const uint4*>(row + 2 * static_cast<int64_t>(k));
+    raw[0] = SMEM_SRC ? *q : __ldg(q);
   } else {
     const uint4* q = reinterpret_cast<const uint4*>(row + 4 * static_cast<int64_t>(k));
-    raw[0] = __ldg(q);
-    raw[1] = __ldg(q + 1);
+    raw[0] = SMEM_SRC ? q[0] : __ldg(q);
+    raw[1] = SMEM_SRC ? q[1] : __ldg(q + 1);
   }
+}
+
+// Block (or named-barrier group) synchronisation used by quant_rows.
+// BAR == 0: __syncthreads; otherwise named barrier BAR over NT threads.
+template <int BAR, int NT>
+__device__ __forceinline__ void group_sync() {
+  if constexpr (BAR == 0)
+    __syncthreads();
+  else
+    asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
+}
+
+// Byte offset of activation k inside a 64-byte chunk row with the 16-byte
+// slots XOR-swizzled by chunk index: lanes that read consecutive chunks hit
+// distinct bank groups.
+__device__ __forceinline__ int xs_swizzle(int k) {
+  const int c = k >> 6, g = (k >> 4) & 3;
+  return (c << 6) | ((g ^ ((c >> 1) & 3)) << 4) | (k & 15);
 }
 
 // Quantise rows 0..M-1 (M <= MT, K % 16 == 0) of x with one CTA of NT
@@ -135,7 +155,7 @@ __device__ __forceinline__ void load8raw(const char* row, int x_dtype, int k, ui
 // writes the codes to dst (row stride dst_stride, generic address) and
 // leaves per-warp partial code sums in S.qpart: the caller's next
 // __syncthreads publishes both.  scale[m] is returned to every thread.
-template <int NT, int MT, int C>
+template <int NT, int MT, int C, bool SMEM_SRC = false, int BAR = 0, bool SWZ = false>
 __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dtype, int64_t row_bytes, int M,
                                            int K, const float* __restrict__ gain, float rms_eps, int8_t* dst,
                                            int64_t dst_stride, QuantScratch<NT, MT>& S, float (&scale)[MT]) {
@@ -169,7 +189,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
         const int k = (c * NT + tid) * 8;
         if (k < K) {
           uint4 raw[2];
-          load8raw(row, x_dtype, k, raw);
+          load8raw<SMEM_SRC>(row, x_dtype, k, raw);
           if (cache_ok) cache[m][c] = raw[0];
           float v[8];
           decode8(raw, x_dtype, v);
@@ -178,7 +198,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
       }
       for (int k = (C * NT + tid) * 8; k < K; k += NT * 8) {
         uint4 raw[2];
-        load8raw(row, x_dtype, k, raw);
+        load8raw<SMEM_SRC>(row, x_dtype, k, raw);
         float v[8];
         decode8(raw, x_dtype, v);
         process(v, k);
@@ -194,7 +214,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
       S.ss[m][warp] = ss[m];
     }
   }
-  __syncthreads();
+  group_sync<BAR, NT>();
   float inv[MT];
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
@@ -236,7 +256,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
           lo |= (static_cast<uint32_t>(q0) & 0xffu) << (8 * i);
           hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);
         }
-        *reinterpret_cast<uint2*>(drow + k) = make_uint2(lo, hi);
+        *reinterpret_cast<uint2*>(drow + (SWZ ? xs_swizzle(k) : k)) = make_uint2(lo, hi);
       };
 #pragma unroll
       for (int c = 0; c < C; ++c) {
@@ -246,7 +266,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
           if (cache_ok)
             raw[0] = cache[m][c];
           else
-            load8raw(row, x_dtype, k, raw);
+            load8raw<SMEM_SRC>(row, x_dtype, k, raw);
           float v[8];
           decode8(raw, x_dtype, v);
           emit(v, k);
@@ -254,7 +274,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
       }
       for (int k = (C * NT + tid) * 8; k < K; k += NT * 8) {
         uint4 raw[2];
-        load8raw(row, x_dtype, k, raw);
+        load8raw<SMEM_SRC>(row, x_dtype, k, raw);
         float v[8];
         decode8(raw, x_dtype, v);
         emit(v, k);

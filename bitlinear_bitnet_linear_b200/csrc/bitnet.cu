@@ -2,13 +2,17 @@
 // argument validation, path selection and kernel launches.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
+#include <new>
+#include <vector>
 #include <mutex>
 
 #include "act.cuh"
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "gemv_stream.cuh"
 #include "weights.cuh"
 
 using namespace bitnet;
@@ -235,6 +239,125 @@ cudaError_t run_gemv(const GemvPlan& pl, cudaStream_t st) {
 }
 
 // ---------------------------------------------------------------------------
+// Streaming GEMV (one or many problems, K % 64 == 0).
+// ---------------------------------------------------------------------------
+struct StreamProblem {
+  const void* x;
+  const uint8_t* Wp;
+  const float* gamma;
+  const float* gain;
+  const float* x_scale;
+  void* y;
+  int32_t* acc;
+  int64_t K, N;
+};
+
+template <int MAXP>
+struct StreamPlan {
+  int MT, R, CW, grid, smem;
+  GsParams<MAXP> p;
+};
+
+template <int MAXP>
+bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int count, int64_t M, int x_dtype,
+                          bool prequant, float rms_eps, int y_dtype, StreamPlan<MAXP>& pl) {
+  if (count < 1 || count > MAXP || M < 1 || M > kGemvMaxM) return BITNET_ERR_UNSUPPORTED;
+  GsParams<MAXP>& p = pl.p;
+  pl.MT = M <= 1 ? 1 : (M <= 2 ? 2 : 4);
+  p.nprob = count;
+  p.M = static_cast<int>(M);
+  p.x_dtype = x_dtype;
+  p.y_dtype = y_dtype;
+  p.prequant = prequant ? 1 : 0;
+  p.rms_eps = rms_eps;
+  int64_t total = 0, max_rowb = 0, max_rows = 0, Kmax = 0, xmax = 0;
+  const int64_t esz = prequant ? 1 : (x_dtype == BITNET_BF16 ? 2 : 4);
+  for (int i = 0; i < count; ++i) {
+    if (pr[i].K % 64 != 0) return BITNET_ERR_UNSUPPORTED;
+    total += pr[i].N * pr[i].K / 4;
+    max_rowb = std::max<int64_t>(max_rowb, pr[i].K / 4);
+    max_rows = std::max<int64_t>(max_rows, pr[i].N);
+    Kmax = std::max<int64_t>(Kmax, pr[i].K);
+    xmax = std::max<int64_t>(xmax, M * pr[i].K * esz);
+  }
+  p.total_bytes = total;
+  // One CTA per SM.  Large streams get a deep ring; small ones (a single
+  // decode call) a footprint small enough that the next call's CTAs fit
+  // beside them (programmatic dependent launch overlaps their weight streams).
+  const bool big = total >= (int64_t(32) << 20);
+  int64_t grid = big ? d->sms : std::min<int64_t>(d->sms, (total + 4095) / 4096);
+  if (grid < 1) grid = 1;
+  pl.grid = static_cast<int>(grid);
+  const int64_t per_cta = (total + grid - 1) / grid;
+  pl.R = pl.MT == 1 ? 4 : (pl.MT == 2 ? 2 : 1);   // largest rows-per-warp task the kernel may pick
+  pl.CW = big ? 16 : 8;
+  p.Kp_max = static_cast<int>(Kmax);
+  const int xs_bytes = pl.MT * p.Kp_max;
+  const int64_t xbuf = (xmax + 127) / 128 * 128;
+  p.nxbuf = (xbuf <= 32 * 1024) ? 2 : 0;
+  p.xbuf_bytes = p.nxbuf ? static_cast<int>(xbuf) : 0;
+  const int budget = big ? d->max_smem_optin : 64 * 1024;
+  int slot = big ? 48 * 1024 : 32 * 1024;
+  if (!big) slot = static_cast<int>(std::min<int64_t>(slot, (per_cta + max_rowb + 15) / 16 * 16));
+  if (slot < max_rowb) slot = static_cast<int>(max_rowb);
+  slot = (slot + 15) / 16 * 16;
+  int room = budget - kGsHeader - xs_bytes - p.nxbuf * p.xbuf_bytes;
+  if (room < slot) room = d->max_smem_optin - kGsHeader - xs_bytes - p.nxbuf * p.xbuf_bytes;
+  int nslots = room / slot;
+  if (nslots > kGsMaxSlots) nslots = kGsMaxSlots;
+  if (!big) nslots = std::min<int64_t>(nslots, std::max<int64_t>(2, (per_cta + slot - 1) / slot + 1));
+  if (nslots < 1) return BITNET_ERR_UNSUPPORTED;
+  p.slot_bytes = slot;
+  p.nslots = nslots;
+  int64_t byte0 = 0;
+  const int unit = pl.CW * pl.R;
+  for (int i = 0; i < count; ++i) {
+    GsProblem& g = p.prob[i];
+    g.x = pr[i].x;
+    g.Wp = pr[i].Wp;
+    g.gamma = pr[i].gamma;
+    g.gain = pr[i].gain;
+    g.x_scale = pr[i].x_scale;
+    g.y = pr[i].y;
+    g.acc = pr[i].acc;
+    g.K = static_cast<int>(pr[i].K);
+    g.N = static_cast<int>(pr[i].N);
+    const int64_t rowb = pr[i].K / 4;
+    int64_t sr = slot / rowb;
+    if (sr >= unit) sr -= sr % unit;
+    g.srows = static_cast<int>(std::max<int64_t>(1, sr));
+    g.pad = 0;
+    g.byte0 = byte0;
+    byte0 += pr[i].N * rowb;
+  }
+  pl.smem = kGsHeader + xs_bytes + p.nxbuf * p.xbuf_bytes + p.nslots * p.slot_bytes;
+  if (pl.smem > d->max_smem_optin) return BITNET_ERR_UNSUPPORTED;
+  return BITNET_OK;
+}
+
+template <int MT, int MAXP, int CW>
+cudaError_t run_stream_t(const StreamPlan<MAXP>& pl, cudaStream_t st) {
+  auto k = gemv_stream_kernel<MT, MAXP, CW>;
+  cudaError_t e = allow_smem(k, pl.smem);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(k, dim3(pl.grid), dim3(CW * 32 + 32), pl.smem, st, pl.p);
+}
+
+template <int MAXP>
+cudaError_t run_stream(const StreamPlan<MAXP>& pl, cudaStream_t st) {
+  const bool wide = pl.CW == 16;
+  switch (pl.MT) {
+    case 1: return wide ? run_stream_t<1, MAXP, 16>(pl, st) : run_stream_t<1, MAXP, 8>(pl, st);
+    case 2: return wide ? run_stream_t<2, MAXP, 16>(pl, st) : run_stream_t<2, MAXP, 8>(pl, st);
+    case 4: return wide ? run_stream_t<4, MAXP, 16>(pl, st) : run_stream_t<4, MAXP, 8>(pl, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+constexpr int kStreamSmallP = 4;
+constexpr int kStreamMaxP = 256;
+
+// ---------------------------------------------------------------------------
 // Tensor-core GEMM launch.
 // ---------------------------------------------------------------------------
 template <int BM, int SS, int AS>
@@ -455,6 +578,21 @@ static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in
   if (path == BITNET_PATH_GEMV && !gemv_ok) return BITNET_ERR_UNSUPPORTED;
   const bool use_gemv = (path == BITNET_PATH_GEMV) || (path == BITNET_PATH_AUTO && gemv_ok);
 
+  if (use_gemv && K % 64 == 0) {
+    StreamProblem sp{x != nullptr ? x : static_cast<const void*>(xq_in), Wp, gamma, rms_gain, scale_in, y, acc, K, N};
+    auto* pl = new (std::nothrow) StreamPlan<kStreamSmallP>;
+    if (pl == nullptr) return BITNET_ERR_CUDA;
+    s = plan_stream<kStreamSmallP>(d, &sp, 1, M, x != nullptr ? x_dtype : BITNET_F32, x == nullptr, rms_eps,
+                                   y != nullptr ? y_dtype : BITNET_F32, *pl);
+    if (s == BITNET_OK) {
+      pl->p.limit_ns = limit;
+      pl->p.status = status;
+    }
+    cudaError_t e = (s == BITNET_OK) ? run_stream<kStreamSmallP>(*pl, st) : cudaSuccess;
+    delete pl;
+    if (s != BITNET_OK) return s;
+    return launch_result(e);
+  }
   if (use_gemv) {
     GemvParams& p = gp.p;
     p.x = x;
@@ -539,6 +677,56 @@ bitnet_status bitnet_linear_q(const int8_t* xq, const float* x_scale, const int3
   if (!aligned16(xq)) return BITNET_ERR_ALIGN;
   return linear_impl(nullptr, BITNET_F32, xq, x_scale, x_sum, M, K, Wp, N, gamma, nullptr, 0.0f, y, y_dtype, acc, ws,
                      ws_bytes, path, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bitnet_status bitnet_linear_grouped(const bitnet_gemv_problem* problems, int count, int64_t M, int x_dtype,
+                                    float rms_eps, int y_dtype, void* ws, size_t ws_bytes, bitnet_stream_t stream) {
+  if (problems == nullptr || ws == nullptr) return BITNET_ERR_NULL;
+  if (count < 1 || count > kStreamMaxP) return BITNET_ERR_SHAPE;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (M < 1 || M > kGemvMaxM) return BITNET_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < kWsHeader) return BITNET_ERR_WORKSPACE;
+  std::vector<StreamProblem> sp(count);
+  for (int i = 0; i < count; ++i) {
+    const bitnet_gemv_problem& q = problems[i];
+    if (q.x == nullptr || q.Wp == nullptr || q.gamma == nullptr || q.y == nullptr) return BITNET_ERR_NULL;
+    bitnet_status s = check_shape(M, q.K, q.N);
+    if (s != BITNET_OK) return s;
+    if (q.K % 64 != 0) return BITNET_ERR_SHAPE;
+    if (!aligned16(q.x) || !aligned16(q.Wp) || !aligned16(q.y) || (q.rms_gain != nullptr && !aligned16(q.rms_gain)))
+      return BITNET_ERR_ALIGN;
+    sp[i] = StreamProblem{q.x, q.Wp, q.gamma, q.rms_gain, nullptr, q.y, nullptr, q.K, q.N};
+  }
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const uint64_t limit = g_limit_ns.load();
+  if (count <= kStreamSmallP) {
+    auto* pl = new (std::nothrow) StreamPlan<kStreamSmallP>;
+    if (pl == nullptr) return BITNET_ERR_CUDA;
+    s = plan_stream<kStreamSmallP>(d, sp.data(), count, M, x_dtype, false, rms_eps, y_dtype, *pl);
+    cudaError_t e = cudaSuccess;
+    if (s == BITNET_OK) {
+      pl->p.limit_ns = limit;
+      pl->p.status = static_cast<uint32_t*>(ws);
+      e = run_stream<kStreamSmallP>(*pl, st);
+    }
+    delete pl;
+    return s != BITNET_OK ? s : launch_result(e);
+  }
+  auto* pl = new (std::nothrow) StreamPlan<kStreamMaxP>;
+  if (pl == nullptr) return BITNET_ERR_CUDA;
+  s = plan_stream<kStreamMaxP>(d, sp.data(), count, M, x_dtype, false, rms_eps, y_dtype, *pl);
+  cudaError_t e = cudaSuccess;
+  if (s == BITNET_OK) {
+    pl->p.limit_ns = limit;
+    pl->p.status = static_cast<uint32_t*>(ws);
+    e = run_stream<kStreamMaxP>(*pl, st);
+  }
+  delete pl;
+  return s != BITNET_OK ? s : launch_result(e);
 }
 
 bitnet_status bitnet_watchdog_selftest(void* ws, size_t ws_bytes, uint32_t limit_us, bitnet_stream_t stream) {

@@ -201,6 +201,33 @@ bitnet_status bitnet_linear_q(const int8_t *xq, const float *x_scale, const int3
                               const float *gamma, void *y, int y_dtype, int32_t *acc,
                               void *ws, size_t ws_bytes, int path, bitnet_stream_t stream);
 
+/* One problem of a grouped GEMV call. */
+typedef struct bitnet_gemv_problem {
+    const void *x;          /* [M, K] activations of the call's x_dtype, device */
+    const uint8_t *Wp;      /* [N, K/4] packed weights (bitnet_pack), device */
+    const float *gamma;     /* device binary32 weight scale */
+    const float *rms_gain;  /* [K] RMSNorm gain, device, or NULL (no norm) */
+    void *y;                /* [M, N] output of the call's y_dtype, device */
+    int64_t K, N;
+} bitnet_gemv_problem;
+
+/* Several independent BitLinear forwards with the same token count M <= 4
+ * in ONE launch: each problem is computed exactly as bitnet_linear would
+ * (quantise its x, contract with its weights, rescale by its gamma), but the
+ * packed weights of all problems are streamed as one contiguous byte range
+ * split evenly over the GPU, so the memory system never idles between calls.
+ * Problems whose x and rms_gain pointers (and K) equal the previous
+ * problem's reuse its quantised activations: fused Q|K|V or up|gate
+ * projections ("Key Technologies ...", Architectural Innovations: BitLinear
+ * layers of one block share their input).  The problems' outputs must not
+ * overlap each other's inputs.
+ * problems: host array of `count` entries (1 <= count <= 256), read during
+ * the call only.  Every K must be a multiple of 64.  ws: at least
+ * bitnet_workspace_bytes(1, 16, 1) bytes (status word only). */
+bitnet_status bitnet_linear_grouped(const bitnet_gemv_problem *problems, int count, int64_t M,
+                                    int x_dtype, float rms_eps, int y_dtype,
+                                    void *ws, size_t ws_bytes, bitnet_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Failure detection.
  * ------------------------------------------------------------------------ */

@@ -300,3 +300,72 @@ def test_no_device_errors_after_suite():
     _, _, g, Wp, x = _prep(300, 2560, 512, seed=4)
     bn.bitnet_linear(x.to(DEV), torch.from_numpy(Wp).to(DEV), torch.tensor([g], device=DEV), ws=ws)
     assert bn.bitnet_get_error(ws) == 0
+
+
+# ---------------------------------------------------------------------------
+# grouped GEMV: many problems in one launch
+# ---------------------------------------------------------------------------
+
+def _grouped_case(specs, M, xd, yd, norm, seed):
+    """specs: list of (K, N, share_x_with_previous)."""
+    problems, refs = [], []
+    x = x_np = None
+    for i, (K, N, share) in enumerate(specs):
+        W = synthetic.latent_weights(N, K, seed + 17 * i)
+        Wq, g = oracle.quant_weights(W.numpy())
+        Wp, _ = oracle.pack(Wq)
+        if not share:
+            x = synthetic.activations(M, K, seed + 31 * i, dtype=xd)
+            x_np = xf32(x)
+            x_dev = x.to(DEV)
+            gain = (torch.from_numpy(np.random.default_rng(seed + i).uniform(0.5, 1.5, K).astype(np.float32))
+                    if norm else None)
+            gain_dev = None if gain is None else gain.to(DEV)
+        y = torch.empty((M, N), dtype=yd, device=DEV)
+        problems.append((x_dev, torch.from_numpy(Wp).to(DEV), torch.tensor([g], dtype=torch.float32, device=DEV),
+                         gain_dev, y))
+        y_ref, *_ = oracle.bitlinear(x_np, Wq, g, None if gain is None else gain.numpy(), 1e-5)
+        refs.append(y_ref)
+    return problems, refs
+
+
+@pytest.mark.parametrize("M", [1, 2, 3, 4])
+@pytest.mark.parametrize("norm", [False, True])
+def test_grouped_small_mixed(M, norm):
+    specs = [(2560, 256, False), (2560, 256, True), (2560, 384, True), (6912, 128, False), (256, 64, False),
+             (2560, 300, False)]
+    problems, refs = _grouped_case(specs, M, torch.bfloat16, torch.bfloat16, norm, seed=40 + M)
+    ws = bn.new_workspace(256)
+    bn.bitnet_linear_grouped(problems, ws=ws)
+    assert bn.bitnet_get_error(ws) == 0
+    for (x, Wp, g, gain, y), y_ref in zip(problems, refs):
+        assert_y(y, y_ref, torch.bfloat16)
+        if not norm:
+            assert (to_np(y.view(torch.int16)).view(np.uint16) == oracle.to_bf16_bits(y_ref)).all()
+
+
+def test_grouped_stack_layer_deep_ring():
+    """One transformer block's seven calls twice (> 32 MB of weights: the
+    deep-ring, one-CTA-per-SM configuration), fp32 in and out."""
+    layer = [(2560, 2560, False), (2560, 2560, True), (2560, 2560, True), (2560, 2560, False),
+             (2560, 6912, False), (2560, 6912, True), (6912, 2560, False)]
+    problems, refs = _grouped_case(layer * 2, 1, torch.float32, torch.float32, False, seed=77)
+    ws = bn.new_workspace(256)
+    bn.bitnet_linear_grouped(problems, ws=ws)
+    assert bn.bitnet_get_error(ws) == 0
+    for (x, Wp, g, gain, y), y_ref in zip(problems, refs):
+        assert (to_np(y) == y_ref).all()
+
+
+def test_grouped_rejects_bad_arguments():
+    x = torch.zeros((1, 96), dtype=torch.bfloat16, device=DEV)      # K % 64 != 0
+    Wp = torch.zeros((8, 24), dtype=torch.uint8, device=DEV)
+    y = torch.zeros((1, 8), dtype=torch.bfloat16, device=DEV)
+    g = torch.ones(1, device=DEV)
+    with pytest.raises(bn.BitnetError) as ei:
+        bn.bitnet_linear_grouped([(x, Wp, g, None, y)])
+    assert ei.value.status == 2
+    x5 = torch.zeros((5, 128), dtype=torch.bfloat16, device=DEV)     # M > 4
+    with pytest.raises(bn.BitnetError):
+        bn.bitnet_linear_grouped([(x5, torch.zeros((8, 32), dtype=torch.uint8, device=DEV), g, None,
+                                   torch.zeros((5, 8), dtype=torch.bfloat16, device=DEV))])

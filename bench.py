@@ -126,16 +126,12 @@ def run_ours(args):
     import torch.distributed as dist
 
     import bitlinear_bitnet_linear_b200 as bn
-    from bitlinear_bitnet_linear_b200 import build, synthetic
+    from bitlinear_bitnet_linear_b200 import build, replicas, synthetic
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local = replicas.rank_info()
     if world > 1:
-        import datetime
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        replicas.init("nccl", timeout_s=120, device=torch.device("cuda", local))
     else:
         torch.cuda.set_device(0)
     dev = torch.device("cuda", torch.cuda.current_device())
@@ -170,7 +166,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     gains = {K: synthetic.unit_gain(K).to(dev) for K in {m.K for m in mats}}
     # inputs of one step: one bf16 activation row per call (independent of the rank's replica)
-    xs_host = [synthetic.activations(1, K, seed=10_000 * (rank + 1) + i, dtype=torch.bfloat16)
+    xs_host = [synthetic.activations(1, K, seed=replicas.replica_seed(i, rank), dtype=torch.bfloat16)
                for i, (K, N, _, _) in enumerate(stack)]
     xs = [x.to(dev) for x in xs_host]
     ys = [torch.empty((1, N), dtype=torch.bfloat16, device=dev) for (K, N, _, _) in stack]
@@ -225,15 +221,12 @@ def run_ours(args):
         if sampler:
             clk = sampler.stop()
         ms_local = e0.elapsed_time(e1) / steps
-        t = torch.tensor([ms_local], device=dev)
-        if world > 1:
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return ms_local, float(t.item()), clk
+        return ms_local, replicas.max_over_ranks(ms_local, dev), clk
 
     graph = capture(step)
     ms, ms_max, clk = time_graph(graph, args.steps, args.warmup, sample_clocks=True)
     assert bn.bitnet_get_error(ws) == 0
-    value = world * bytes_step / (ms_max * 1e-3) / 1e9
+    value = replicas.whole_job_rate(bytes_step, world, ms_max * 1e-3) / 1e9
     per_rank = bytes_step / (ms * 1e-3) / 1e9
 
     # ---- the same 210 calls as a dependent chain of separate launches ------
@@ -289,12 +282,9 @@ def run_ours(args):
                 e2e_step()
             e1.record(stream)
         barrier()
-        ems = e0.elapsed_time(e1) / e2e_steps
-        te = torch.tensor([ems], device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": round(world * bytes_step / (float(te.item()) * 1e-3) / 1e9, 2), "unit": "GB/s",
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(float(te.item()), 4),
+        ems = replicas.max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
+        e2e = {"value": round(replicas.whole_job_rate(bytes_step, world, ems * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ems, 4),
                "path": "python binding -> C ABI bitnet_linear_grouped (210 problems), pinned host x in, y out"}
 
     # ---- prefill GEMM (secondary) ------------------------------------------

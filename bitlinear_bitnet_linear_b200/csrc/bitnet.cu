@@ -290,14 +290,16 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
   pl.grid = static_cast<int>(grid);
   const int64_t per_cta = (total + grid - 1) / grid;
   pl.R = pl.MT == 1 ? 4 : (pl.MT == 2 ? 2 : 1);   // largest rows-per-warp task the kernel may pick
-  pl.CW = big ? 16 : 8;
+  // eight consumer warps: two rounds of their 10 KB tasks fit in the ring
+  pl.CW = 8;
+  p.deep = big ? 1 : 0;
   p.Kp_max = static_cast<int>(Kmax);
   const int xs_bytes = pl.MT * p.Kp_max;
   const int64_t xbuf = (xmax + 127) / 128 * 128;
   p.nxbuf = (xbuf <= 32 * 1024) ? 2 : 0;
   p.xbuf_bytes = p.nxbuf ? static_cast<int>(xbuf) : 0;
   const int budget = big ? d->max_smem_optin : 64 * 1024;
-  int slot = big ? 48 * 1024 : 32 * 1024;
+  int slot = big ? 40 * 1024 : 32 * 1024;
   if (!big) slot = static_cast<int>(std::min<int64_t>(slot, (per_cta + max_rowb + 15) / 16 * 16));
   if (slot < max_rowb) slot = static_cast<int>(max_rowb);
   slot = (slot + 15) / 16 * 16;
@@ -324,7 +326,13 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
     g.N = static_cast<int>(pr[i].N);
     const int64_t rowb = pr[i].K / 4;
     int64_t sr = slot / rowb;
-    if (sr >= unit) sr -= sr % unit;
+    // stage rows aligned to the consumers' task size (16 rows for the 8-lane
+    // group path, 4 for the warp path)
+    const bool lg = pl.MT == 1 && pr[i].K <= 4096 && (pr[i].K / 16) % 8 == 0;
+    const int64_t task = big ? (lg ? 8 : 4) : (lg ? 16 : 4);
+    if (sr >= task) sr -= sr % task;
+    if (big && lg && sr > 8 * pl.CW) sr = 8 * pl.CW;   // one 8-row task per warp per stage
+    (void)unit;
     g.srows = static_cast<int>(std::max<int64_t>(1, sr));
     g.pad = 0;
     g.byte0 = byte0;
@@ -335,21 +343,21 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
   return BITNET_OK;
 }
 
-template <int MT, int MAXP, int CW>
+template <int MT, int MAXP, bool DEEP>
 cudaError_t run_stream_t(const StreamPlan<MAXP>& pl, cudaStream_t st) {
-  auto k = gemv_stream_kernel<MT, MAXP, CW>;
+  auto k = gemv_stream_kernel<MT, MAXP, 8, DEEP>;
   cudaError_t e = allow_smem(k, pl.smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k, dim3(pl.grid), dim3(CW * 32 + 32), pl.smem, st, pl.p);
+  return launch_pdl(k, dim3(pl.grid), dim3(8 * 32 + 32), pl.smem, st, pl.p);
 }
 
 template <int MAXP>
 cudaError_t run_stream(const StreamPlan<MAXP>& pl, cudaStream_t st) {
-  const bool wide = pl.CW == 16;
+  const bool deep = pl.p.deep != 0;
   switch (pl.MT) {
-    case 1: return wide ? run_stream_t<1, MAXP, 16>(pl, st) : run_stream_t<1, MAXP, 8>(pl, st);
-    case 2: return wide ? run_stream_t<2, MAXP, 16>(pl, st) : run_stream_t<2, MAXP, 8>(pl, st);
-    case 4: return wide ? run_stream_t<4, MAXP, 16>(pl, st) : run_stream_t<4, MAXP, 8>(pl, st);
+    case 1: return deep ? run_stream_t<1, MAXP, true>(pl, st) : run_stream_t<1, MAXP, false>(pl, st);
+    case 2: return deep ? run_stream_t<2, MAXP, true>(pl, st) : run_stream_t<2, MAXP, false>(pl, st);
+    case 4: return deep ? run_stream_t<4, MAXP, true>(pl, st) : run_stream_t<4, MAXP, false>(pl, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -488,7 +496,7 @@ bitnet_status bitnet_quant_weights(const float* W, int64_t N, int64_t K, float e
   uint32_t* status = static_cast<uint32_t*>(ws);
   uint64_t* partial = reinterpret_cast<uint64_t*>(static_cast<uint8_t*>(ws) + kWsHeader);
   absmean_partial_kernel<<<static_cast<unsigned>(blocks), kAbsThreads, 0, st>>>(W, n, per_block, partial, status);
-  absmean_finalize_kernel<<<1, 32, 0, st>>>(partial, static_cast<int>(blocks), n, gamma);
+  absmean_finalize_kernel<<<1, kAbsFinThreads, 0, st>>>(partial, static_cast<int>(blocks), n, gamma);
   if (Wq != nullptr) {
     ternarise_kernel<<<elementwise_grid(n / 4, d), 256, 0, st>>>(W, n / 4, gamma, eps, Wq);
   }

@@ -35,6 +35,7 @@ constexpr int kGsMaxSlots = 12;
 constexpr int kGsMaxX = 2;
 constexpr int kGsHeader = 2048;
 constexpr int kGsBar = 1;          // named barrier of the consumer warps
+constexpr int kGsPrefetch = 12;    // weight stages pulled into L2 ahead of the ring
 
 struct GsProblem {
   const void* x;          // [M, K] raw activations (x_dtype) or int8 codes (prequant)
@@ -60,6 +61,7 @@ struct GsParams {
   int slot_bytes, nslots;        // weight ring
   int xbuf_bytes, nxbuf;         // activation ring (nxbuf == 0: read x from global memory)
   int Kp_max;                    // int8 code rows in shared memory, K rounded up to 64
+  int deep;                      // 1: long stream (tasks flow across stages), 0: one short call
   uint64_t limit_ns;
   uint32_t* status;
 };
@@ -92,65 +94,146 @@ __device__ __forceinline__ void gs_cta_start(const GsParams<MAXP>& p, int b, int
   row = 0;
 }
 
-// Contract the rows of one weight stage (rc rows starting at problem row r)
-// against the shared-memory activation codes; warps take groups of R rows,
-// lane l takes code words l, l + 32, ... of those rows.
-template <int R, int MT, int CW>
-__device__ __forceinline__ void gs_contract(const uint8_t* buf, int rc, int rowwords, int nword, const int8_t* xs,
-                                            int Kp, int warp, int lane, const int (&xsum)[MT],
-                                            const float (&sc)[MT], float gamma, const GsProblem& P, int r, int M,
-                                            int y_dtype) {
-  for (int rg = warp; rg * R < rc; rg += CW) {
-    const int nr = min(R, rc - rg * R);
-    int a[R][MT][4];
+// Short rows (M = 1, K <= 4096): a warp is four 8-lane groups, each owning
+// RS consecutive rows; a lane walks every eighth code word of its rows, so a
+// row's partial sums are reduced over 8 lanes (3 shuffles).  The groups start
+// their walks 8 words apart (rotation modulo the row length), so rows whose
+// word count is a multiple of 32 do not collide on shared-memory banks.
+// Rows [row0, row0 + 4 RS) of the stage; requires nword % 8 == 0.
+template <int RS>
+__device__ __forceinline__ void gs_task_lanegroups(const uint32_t* wbase, int rc, int row0, int rowwords, int nword,
+                                                   const int8_t* xs, int lane, int xsum0, float gs0,
+                                                   const GsProblem& P, int r, int y_dtype) {
+  const int lg = lane >> 3, lj = lane & 7;
+  const int rb = row0 + lg * RS;                 // this group's first row
+  const int nr = max(0, min(RS, rc - rb));
+  int a[RS][4];
 #pragma unroll
-    for (int i = 0; i < R; ++i)
+  for (int i = 0; i < RS; ++i)
 #pragma unroll
-      for (int m = 0; m < MT; ++m)
+    for (int f = 0; f < 4; ++f) a[i][f] = 0;
+  const uint32_t* wb = wbase + static_cast<int64_t>(rb) * rowwords;
+  int g = lj + 8 * lg;
+  if (g >= nword) g -= nword * (g / nword);
+  if (nr == RS) {
+#pragma unroll 4
+    for (int t = 0; t < nword; t += 8) {
+      uint32_t w[RS];
 #pragma unroll
-        for (int f = 0; f < 4; ++f) a[i][m][f] = 0;
-    const uint32_t* wb = reinterpret_cast<const uint32_t*>(buf) + (rg * R) * rowwords;
-    // 16 weights (one code word) against the 16 activations at bytes [16 g, 16 g + 16)
-#pragma unroll 2
+      for (int i = 0; i < RS; ++i) w[i] = wb[i * rowwords + g];
+      const uint4 xv = *reinterpret_cast<const uint4*>(xs + 16 * g);
+#pragma unroll
+      for (int i = 0; i < RS; ++i) {
+        a[i][0] = dp4a_us(w[i] & 0x03030303u, xv.x, a[i][0]);
+        a[i][1] = dp4a_us(w[i] & 0x0C0C0C0Cu, xv.y, a[i][1]);
+        a[i][2] = dp4a_us(w[i] & 0x30303030u, xv.z, a[i][2]);
+        a[i][3] = dp4a_us(w[i] & 0xC0C0C0C0u, xv.w, a[i][3]);
+      }
+      g += 8;
+      if (g >= nword) g -= nword;
+    }
+  } else if (nr > 0) {
+    for (int t = 0; t < nword; t += 8) {
+      uint32_t w[RS];
+#pragma unroll
+      for (int i = 0; i < RS; ++i) w[i] = (i < nr) ? wb[i * rowwords + g] : 0u;
+      const uint4 xv = *reinterpret_cast<const uint4*>(xs + 16 * g);
+#pragma unroll
+      for (int i = 0; i < RS; ++i) {
+        a[i][0] = dp4a_us(w[i] & 0x03030303u, xv.x, a[i][0]);
+        a[i][1] = dp4a_us(w[i] & 0x0C0C0C0Cu, xv.y, a[i][1]);
+        a[i][2] = dp4a_us(w[i] & 0x30303030u, xv.z, a[i][2]);
+        a[i][3] = dp4a_us(w[i] & 0xC0C0C0C0u, xv.w, a[i][3]);
+      }
+      g += 8;
+      if (g >= nword) g -= nword;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < RS; ++i) {
+    int t = a[i][0] + (a[i][1] >> 2) + (a[i][2] >> 4) + (a[i][3] >> 6);
+    t += __shfl_xor_sync(0xffffffffu, t, 4);
+    t += __shfl_xor_sync(0xffffffffu, t, 2);
+    t += __shfl_xor_sync(0xffffffffu, t, 1);
+    a[i][0] = t;
+  }
+#pragma unroll
+  for (int i = 0; i < RS; ++i) {
+    if (lj == i && i < nr) {
+      const int64_t n = r + rb + i;
+      const int accv = a[i][0] - xsum0;
+      if (P.acc != nullptr) P.acc[n] = accv;
+      if (P.y != nullptr) store_y(P.y, y_dtype, n, __fmul_rn(__int2float_rn(accv), gs0));
+    }
+  }
+}
+
+// Long rows or M > 1: a warp owns R rows, lane l walks code words l, l + 32, ...
+// Rows [row0, row0 + R) of the stage.
+template <int R, int MT>
+__device__ __forceinline__ void gs_task_warp(const uint32_t* wbase, int rc, int row0, int rowwords, int nword,
+                                             const int8_t* xs, int Kp, int lane, const int (&xsum)[MT],
+                                             const float (&sc)[MT], float gamma, const GsProblem& P, int r, int M,
+                                             int y_dtype) {
+  const int nr = min(R, rc - row0);
+  int a[R][MT][4];
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+      for (int f = 0; f < 4; ++f) a[i][m][f] = 0;
+  const uint32_t* wb = wbase + static_cast<int64_t>(row0) * rowwords;
+  auto body = [&](const uint32_t (&w)[R], int g) {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      const uint4 xv = *reinterpret_cast<const uint4*>(xs + m * Kp + 16 * g);
+#pragma unroll
+      for (int i = 0; i < R; ++i) {
+        a[i][m][0] = dp4a_us(w[i] & 0x03030303u, xv.x, a[i][m][0]);
+        a[i][m][1] = dp4a_us(w[i] & 0x0C0C0C0Cu, xv.y, a[i][m][1]);
+        a[i][m][2] = dp4a_us(w[i] & 0x30303030u, xv.z, a[i][m][2]);
+        a[i][m][3] = dp4a_us(w[i] & 0xC0C0C0C0u, xv.w, a[i][m][3]);
+      }
+    }
+  };
+  if (nr == R) {
+#pragma unroll 4
+    for (int g = lane; g < nword; g += 32) {
+      uint32_t w[R];
+#pragma unroll
+      for (int i = 0; i < R; ++i) w[i] = wb[i * rowwords + g];
+      body(w, g);
+    }
+  } else {
     for (int g = lane; g < nword; g += 32) {
       uint32_t w[R];
 #pragma unroll
       for (int i = 0; i < R; ++i) w[i] = (i < nr) ? wb[i * rowwords + g] : 0u;
+      body(w, g);
+    }
+  }
 #pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        const uint4 xv = *reinterpret_cast<const uint4*>(xs + m * Kp + 16 * g);
+  for (int i = 0; i < R; ++i)
 #pragma unroll
-        for (int i = 0; i < R; ++i) {
-          a[i][m][0] = dp4a_us(w[i] & 0x03030303u, xv.x, a[i][m][0]);
-          a[i][m][1] = dp4a_us(w[i] & 0x0C0C0C0Cu, xv.y, a[i][m][1]);
-          a[i][m][2] = dp4a_us(w[i] & 0x30303030u, xv.z, a[i][m][2]);
-          a[i][m][3] = dp4a_us(w[i] & 0xC0C0C0C0u, xv.w, a[i][m][3]);
-        }
+    for (int m = 0; m < MT; ++m)
+      a[i][m][0] = warp_sum(a[i][m][0] + (a[i][m][1] >> 2) + (a[i][m][2] >> 4) + (a[i][m][3] >> 6));
+#pragma unroll
+  for (int i = 0; i < R; ++i)
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if (lane == i * MT + m && i < nr && m < M) {
+        const int64_t n = r + row0 + i;
+        const int accv = a[i][m][0] - xsum[m];
+        const int64_t idx = static_cast<int64_t>(m) * P.N + n;
+        if (P.acc != nullptr) P.acc[idx] = accv;
+        if (P.y != nullptr) store_y(P.y, y_dtype, idx, __fmul_rn(__int2float_rn(accv), __fmul_rn(gamma, sc[m])));
       }
     }
-    // field f holds 4^f times its sum: exact shifts, then the lane reduction
-#pragma unroll
-    for (int i = 0; i < R; ++i)
-#pragma unroll
-      for (int m = 0; m < MT; ++m)
-        a[i][m][0] = warp_sum(a[i][m][0] + (a[i][m][1] >> 2) + (a[i][m][2] >> 4) + (a[i][m][3] >> 6));
-#pragma unroll
-    for (int i = 0; i < R; ++i)
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        if (lane == i * MT + m && i < nr && m < M) {
-          const int64_t n = r + rg * R + i;
-          const int accv = a[i][m][0] - xsum[m];
-          const int64_t idx = static_cast<int64_t>(m) * P.N + n;
-          if (P.acc != nullptr) P.acc[idx] = accv;
-          if (P.y != nullptr) store_y(P.y, y_dtype, idx, __fmul_rn(__int2float_rn(accv), __fmul_rn(gamma, sc[m])));
-        }
-      }
-  }
 }
 
 // CW consumer warps + one producer warp.
-template <int MT, int MAXP, int CW>
+template <int MT, int MAXP, int CW, bool DEEP>
 __global__ void __launch_bounds__(CW * 32 + 32, (CW <= 8 ? 2 : 1))
     gemv_stream_kernel(const __grid_constant__ GsParams<MAXP> p) {
   constexpr int kGsConsumers = CW * 32;
@@ -208,6 +291,28 @@ __global__ void __launch_bounds__(CW * 32 + 32, (CW <= 8 ? 2 : 1))
       int u = 0;          // activation buffers issued
       bool dep_waited = false;
       bool ok = true;
+      // L2 prefetch cursor: walks the same stage sequence kGsPrefetch stages
+      // ahead of the shared-memory copies, so those copies hit in L2 and the
+      // DRAM stream does not wait for ring slots to be released.
+      int pq = pb, pr = (pb <= qlast) ? rb : 0, npf = 0;
+      auto prefetch_upto = [&](int upto) {
+        while (npf < upto && pq <= qlast) {
+          int q0, q1;
+          seg_bounds(pq, q0, q1);
+          if (pr >= q1) {
+            ++pq;
+            if (pq <= qlast) seg_bounds(pq, pr, q1);
+            continue;
+          }
+          const GsProblem& Q = p.prob[pq];
+          const int64_t qrowb = Q.K / 4;
+          const int rc = min(Q.srows, q1 - pr);
+          bulk_prefetch_l2(Q.Wp + static_cast<int64_t>(pr) * qrowb, static_cast<uint32_t>(rc * qrowb));
+          pr += Q.srows;
+          ++npf;
+        }
+      };
+      prefetch_upto(kGsPrefetch);
       // Phase 1: fill the weight ring before the dependency wait.
       {
         int issued = 0;
@@ -222,6 +327,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, (CW <= 8 ? 2 : 1))
             mbar_expect_tx(&H.wfull[issued], bytes);
             bulk_g2s(wring + issued * p.slot_bytes, P.Wp + static_cast<int64_t>(r) * rowb, bytes, &H.wfull[issued]);
             ++issued;
+            prefetch_upto(issued + kGsPrefetch);
           }
         }
         t = issued;
@@ -263,6 +369,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, (CW <= 8 ? 2 : 1))
           mbar_expect_tx(&H.wfull[s], bytes);
           bulk_g2s(wring + s * p.slot_bytes, P.Wp + static_cast<int64_t>(r) * rowb, bytes, &H.wfull[s]);
           ++t;
+          prefetch_upto(t + kGsPrefetch);
         }
       }
       if (!dep_waited) {
@@ -293,6 +400,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, (CW <= 8 ? 2 : 1))
     xsum[m] = 0;
   }
   int ts = 0, u = 0;
+  int64_t task0 = 0;
   bool triggered = false;
   for (int q = pb; q <= qlast; ++q) {
     int r0, r1;
@@ -372,37 +480,77 @@ __global__ void __launch_bounds__(CW * 32 + 32, (CW <= 8 ? 2 : 1))
     const int64_t rowb = P.K / 4;
     const int nword = P.K / 16;      // 32-bit code words (16 weights) per row
     const int rowwords = static_cast<int>(rowb / 4);
+    // Work units ("tasks") of every stage are numbered globally and dealt to
+    // the warps round-robin, so a warp with nothing to do in one stage moves
+    // on to the next; a slot is released when every warp has passed it.
+    const bool lanegroups = (MT == 1) && (P.K <= 4096) && (nword % 8 == 0);
+    const float gs0 = __fmul_rn(gamma, sc[0]);
     for (int r = r0; r < r1; r += P.srows, ++ts) {
       const int s = ts % p.nslots;
+      const int rc = min(P.srows, r1 - r);
+      // task size for this stage (identical in every warp): the largest that
+      // still gives every warp work, up to 16 rows (4 per 8-lane group) or 4
+      // rows per warp
+      int kind, rows_per_task;
+      if constexpr (DEEP) {
+        // long streams: fixed task sizes (8-row lane-group tasks; 4/2/1-row
+        // warp tasks by M); stages hold one task per warp
+        kind = lanegroups ? 2 : (MT == 1 ? 4 : (MT == 2 ? 2 : 1));
+        rows_per_task = lanegroups ? 4 * kind : kind;
+      } else if (lanegroups) {
+        kind = ((rc + 15) / 16 >= kGsWarps) ? 4 : 1;
+        rows_per_task = 4 * kind;
+      } else {
+        auto cost = [&](int RR) { return ((rc + RR - 1) / RR + kGsWarps - 1) / kGsWarps * RR; };
+        kind = 1;
+        if (MT <= 2 && cost(2) <= cost(1)) kind = 2;
+        if (MT == 1 && cost(4) <= cost(kind)) kind = 4;
+        rows_per_task = kind;
+      }
+      const int nt = (rc + rows_per_task - 1) / rows_per_task;
+      const int j0 = (warp - static_cast<int>(task0 % kGsWarps) + kGsWarps) % kGsWarps;
+      // Every warp waits for every stage to land, even one with no task in
+      // it, before releasing it: a warp is then never more than one phase of
+      // a slot ahead of the others, which keeps the parity waits and the
+      // release counts of each slot's barriers exact.
       const bool got = mbar_wait_bounded(&H.wfull[s], (ts / p.nslots) & 1, p.limit_ns, abort_flag);
       if (!got && !*abort_flag) {
         record_error(p.status, BITNET_ERR_TIMEOUT, 0x403u);
         *abort_flag = 1;
       }
-      const int rc = min(P.srows, r1 - r);
-      const uint8_t* buf = wring + s * p.slot_bytes;
-      if (got) {
-        // rows per warp task: the smallest critical path (rounds of warp
-        // tasks x rows per task), ties to the larger task, which reuses each
-        // activation word across more rows
-        auto cost = [&](int RR) { return ((rc + RR - 1) / RR + CW - 1) / CW * RR; };
-        if constexpr (MT == 1) {
-          const int c1 = cost(1), c2 = cost(2), c4 = cost(4);
-          if (c4 <= c2 && c4 <= c1)
-            gs_contract<4, MT, CW>(buf, rc, rowwords, nword, xs, Kp, warp, lane, xsum, sc, gamma, P, r, p.M, p.y_dtype);
-          else if (c2 <= c1)
-            gs_contract<2, MT, CW>(buf, rc, rowwords, nword, xs, Kp, warp, lane, xsum, sc, gamma, P, r, p.M, p.y_dtype);
-          else
-            gs_contract<1, MT, CW>(buf, rc, rowwords, nword, xs, Kp, warp, lane, xsum, sc, gamma, P, r, p.M, p.y_dtype);
-        } else if constexpr (MT == 2) {
-          if (cost(2) <= cost(1))
-            gs_contract<2, MT, CW>(buf, rc, rowwords, nword, xs, Kp, warp, lane, xsum, sc, gamma, P, r, p.M, p.y_dtype);
-          else
-            gs_contract<1, MT, CW>(buf, rc, rowwords, nword, xs, Kp, warp, lane, xsum, sc, gamma, P, r, p.M, p.y_dtype);
-        } else {
-          gs_contract<1, MT, CW>(buf, rc, rowwords, nword, xs, Kp, warp, lane, xsum, sc, gamma, P, r, p.M, p.y_dtype);
+      if (j0 < nt) {
+        if (got) {
+          const uint32_t* wbase = reinterpret_cast<const uint32_t*>(wring + s * p.slot_bytes);
+          for (int j = j0; j < nt; j += kGsWarps) {
+            const int row0 = j * rows_per_task;
+            if (lanegroups) {
+              if constexpr (DEEP) {
+                gs_task_lanegroups<2>(wbase, rc, row0, rowwords, nword, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+              } else {
+                if (kind == 4)
+                  gs_task_lanegroups<4>(wbase, rc, row0, rowwords, nword, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+                else
+                  gs_task_lanegroups<1>(wbase, rc, row0, rowwords, nword, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+              }
+            } else if constexpr (DEEP) {
+              gs_task_warp<(MT == 1 ? 4 : (MT == 2 ? 2 : 1)), MT>(wbase, rc, row0, rowwords, nword, xs, Kp, lane, xsum,
+                                                                   sc, gamma, P, r, p.M, p.y_dtype);
+            } else if (kind == 4) {
+              if constexpr (MT == 1)
+                gs_task_warp<4, MT>(wbase, rc, row0, rowwords, nword, xs, Kp, lane, xsum, sc, gamma, P, r, p.M,
+                                    p.y_dtype);
+            } else if (kind == 2) {
+              if constexpr (MT <= 2)
+                gs_task_warp<2, MT>(wbase, rc, row0, rowwords, nword, xs, Kp, lane, xsum, sc, gamma, P, r, p.M,
+                                    p.y_dtype);
+            } else {
+              gs_task_warp<1, MT>(wbase, rc, row0, rowwords, nword, xs, Kp, lane, xsum, sc, gamma, P, r, p.M,
+                                  p.y_dtype);
+            }
+          }
         }
       }
+      task0 += nt;
       __syncwarp();
       if (lane == 0) mbar_arrive(&H.wempty[s]);
     }

@@ -73,21 +73,35 @@ __global__ void __launch_bounds__(kAbsThreads) absmean_partial_kernel(const floa
   }
 }
 
-// One warp: sum the per-block bins, assemble the exact total in a 384-bit
-// integer (units of 2^-150), round it once to binary64, divide by n in
-// binary64 and round to binary32.
-__global__ void absmean_finalize_kernel(const uint64_t* __restrict__ partial, int nblocks, int64_t n,
-                                        float* __restrict__ gamma_out) {
+// 256 threads: sum the per-block bins (16 threads per bin, exact in 128
+// bits), then one thread assembles the exact total in a 384-bit integer
+// (units of 2^-150), rounds it once to binary64, divides by n in binary64 and
+// rounds to binary32.
+constexpr int kAbsFinThreads = 256;
+__global__ void __launch_bounds__(kAbsFinThreads) absmean_finalize_kernel(const uint64_t* __restrict__ partial,
+                                                                          int nblocks, int64_t n,
+                                                                          float* __restrict__ gamma_out) {
+  __shared__ unsigned long long plo[16][kAbsBins], phi[16][kAbsBins];
   __shared__ unsigned long long lo_s[kAbsBins], hi_s[kAbsBins];
-  const int lane = threadIdx.x;
-  if (lane < kAbsBins) {
+  const int tid = threadIdx.x;
+  {
+    const int bin = tid & (kAbsBins - 1), part = tid >> 4;
     unsigned __int128 s = 0;
-    for (int b = 0; b < nblocks; ++b) s += partial[static_cast<int64_t>(b) * kAbsBins + lane];
-    lo_s[lane] = static_cast<unsigned long long>(s);
-    hi_s[lane] = static_cast<unsigned long long>(s >> 64);
+    for (int b = part; b < nblocks; b += kAbsFinThreads / kAbsBins)
+      s += partial[static_cast<int64_t>(b) * kAbsBins + bin];
+    plo[part][bin] = static_cast<unsigned long long>(s);
+    phi[part][bin] = static_cast<unsigned long long>(s >> 64);
   }
-  __syncwarp();
-  if (lane != 0) return;
+  __syncthreads();
+  if (tid < kAbsBins) {
+    unsigned __int128 s = 0;
+    for (int part = 0; part < kAbsFinThreads / kAbsBins; ++part)
+      s += (static_cast<unsigned __int128>(phi[part][tid]) << 64) | plo[part][tid];
+    lo_s[tid] = static_cast<unsigned long long>(s);
+    hi_s[tid] = static_cast<unsigned long long>(s >> 64);
+  }
+  __syncthreads();
+  if (tid != 0) return;
 
   uint64_t limb[6] = {0, 0, 0, 0, 0, 0};
   for (int b = 0; b < kAbsBins; ++b) {

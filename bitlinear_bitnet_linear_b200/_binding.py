@@ -26,8 +26,8 @@ PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
 EXPORTS = ("bitnet_workspace_bytes", "bitnet_quant_weights_workspace_bytes", "bitnet_workspace_init",
            "bitnet_get_error", "bitnet_status_str", "bitnet_quant_weights", "bitnet_ternarise",
            "bitnet_pack", "bitnet_unpack", "bitnet_quant_act", "bitnet_linear", "bitnet_linear_ex",
-           "bitnet_linear_q", "bitnet_linear_grouped", "bitnet_set_wait_limit_us",
-           "bitnet_watchdog_selftest")
+           "bitnet_linear_q", "bitnet_linear_grouped", "bitnet_quant_weights_noalloc",
+           "bitnet_set_wait_limit_us", "bitnet_watchdog_selftest")
 
 
 class GemvProblem(ctypes.Structure):
@@ -64,6 +64,7 @@ def lib() -> ctypes.CDLL:
         "bitnet_status_str": ([I32], ctypes.c_char_p),
         "bitnet_quant_weights": ([P, I64, I64, F, P, P, P, SZ, P], I32),
         "bitnet_ternarise": ([P, I64, I64, P, F, P, P], I32),
+        "bitnet_quant_weights_noalloc": ([P, I64, I64, F, P, P, P], I32),
         "bitnet_pack": ([P, I64, I64, P, P, P], I32),
         "bitnet_unpack": ([P, I64, I64, P, P, P], I32),
         "bitnet_quant_act": ([P, I32, I64, I64, P, F, P, P, P, P], I32),
@@ -174,6 +175,27 @@ def bitnet_quant_weights(W: torch.Tensor, eps: float = 1e-8, Wq: torch.Tensor | 
         ws = new_workspace(bitnet_quant_weights_workspace_bytes(N, K), W.device)
     _check(lib().bitnet_quant_weights(_ptr(W), N, K, float(eps), _ptr(Wq) if want_wq else None, _ptr(gamma),
                                       _ptr(ws), ws.numel(), _stream(stream)), "bitnet_quant_weights")
+    return Wq, gamma
+
+
+# Largest N*K bitnet_quant_weights_noalloc accepts: 2048 blocks of 2^24 weights.
+NOALLOC_MAX_ELEMENTS = 2048 * (1 << 24)
+
+
+def bitnet_quant_weights_noalloc(W: torch.Tensor, eps: float = 1e-8, Wq: torch.Tensor | None = None,
+                                 gamma: torch.Tensor | None = None, want_wq: bool = True, stream=None):
+    """bitnet_quant_weights without a workspace (the library's own scratch).
+    Outputs are allocated here only when not given."""
+    N, K = W.shape
+    if N * K > NOALLOC_MAX_ELEMENTS:
+        raise BitnetError(2, f"bitnet_quant_weights_noalloc: N*K = {N * K} exceeds the scratch limit "
+                             f"{NOALLOC_MAX_ELEMENTS} (use bitnet_quant_weights with a workspace)")
+    if want_wq and Wq is None:
+        Wq = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    if gamma is None:
+        gamma = torch.empty(1, dtype=torch.float32, device=W.device)
+    _check(lib().bitnet_quant_weights_noalloc(_ptr(W), N, K, float(eps), _ptr(Wq) if want_wq else None,
+                                              _ptr(gamma), _stream(stream)), "bitnet_quant_weights_noalloc")
     return Wq, gamma
 
 

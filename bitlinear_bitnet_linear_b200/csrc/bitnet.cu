@@ -405,6 +405,15 @@ bitnet_status launch_result(cudaError_t e) {
   return e == cudaSuccess ? BITNET_OK : BITNET_ERR_CUDA;
 }
 
+// Scratch of bitnet_quant_weights_noalloc: the per-block exact-sum bins.
+// Every GPU that loads the library holds these 256 KiB until exit.
+constexpr int kNoAllocMaxBlocks = 2048;
+static __device__ __align__(256) uint64_t g_noalloc_scratch[kNoAllocMaxBlocks * kAbsBins];
+
+// Device address of the scratch array per device, resolved once with that
+// device current (the host symbol itself is not a device address).
+uint64_t* g_noalloc_ptr[kMaxDevices] = {};
+
 }  // namespace
 
 // ===========================================================================
@@ -748,4 +757,53 @@ bitnet_status bitnet_watchdog_selftest(void* ws, size_t ws_bytes, uint32_t limit
   return launch_result(cudaSuccess);
 }
 
+// Variant of bitnet_quant_weights that allocates nothing: its scratch is the
+// file-scope array above instead of a caller workspace.
+bitnet_status bitnet_quant_weights_noalloc(const float* W, int64_t N, int64_t K, float eps, int8_t* Wq,
+                                           float* gamma, bitnet_stream_t stream) {
+  if (W == nullptr || gamma == nullptr) return BITNET_ERR_NULL;
+  if (check_shape(1, K, N) != BITNET_OK) return BITNET_ERR_SHAPE;
+  if (!aligned16(W) || (Wq != nullptr && !aligned16(Wq))) return BITNET_ERR_ALIGN;
+  // the scratch holds kNoAllocMaxBlocks blocks of at most kAbsMaxPerBlock elements
+  if (N * K > static_cast<int64_t>(kNoAllocMaxBlocks) * kAbsMaxPerBlock) return BITNET_ERR_SHAPE;
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return BITNET_ERR_CUDA;
+  }
+  uint64_t* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+        cudaGetLastError();
+        return BITNET_ERR_CUDA;
+      }
+      g_noalloc_ptr[dev] = static_cast<uint64_t*>(ptr);
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  const int64_t n = N * K;
+  // same partition rule as bitnet_quant_weights, capped by the scratch size
+  int64_t blocks = (n + kAbsMaxPerBlock - 1) / kAbsMaxPerBlock;
+  const int64_t want = static_cast<int64_t>(d->sms) * 8;
+  if (blocks < want) blocks = want;
+  if (blocks > kNoAllocMaxBlocks) blocks = kNoAllocMaxBlocks;
+  int64_t per_block = (n + blocks - 1) / blocks;
+  per_block = (per_block + 15) / 16 * 16;   // <= kAbsMaxPerBlock by the size check above
+  blocks = (n + per_block - 1) / per_block;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  absmean_partial_kernel<<<static_cast<unsigned>(blocks), kAbsThreads, 0, st>>>(W, n, per_block, scratch, nullptr);
+  absmean_finalize_kernel<<<1, kAbsFinThreads, 0, st>>>(scratch, static_cast<int>(blocks), n, gamma);
+  if (Wq != nullptr) {
+    ternarise_kernel<<<elementwise_grid(n / 4, d), 256, 0, st>>>(W, n / 4, gamma, eps, Wq);
+  }
+  return launch_result(cudaSuccess);
+}
+
 }  // extern "C"
+

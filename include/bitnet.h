@@ -228,6 +228,27 @@ bitnet_status bitnet_linear_grouped(const bitnet_gemv_problem *problems, int cou
                                     int x_dtype, float rms_eps, int y_dtype,
                                     void *ws, size_t ws_bytes, bitnet_stream_t stream);
 
+/* bitnet_quant_weights for callers that cannot allocate device memory and
+ * so cannot provide its workspace: code running under CUDA stream capture
+ * (where allocation is not allowed), or a host framework that owns the
+ * device memory pool and gives extensions no allocator.  Same arguments and
+ * results as bitnet_quant_weights (gamma and W_q are identical), minus the
+ * workspace.  The pages have no counterpart: this is an interface choice.
+ *   - Scratch: a 256 KiB array inside the library, resident on every GPU
+ *     that loads it until the process exits.  Nothing is allocated or freed.
+ *   - Limit: N*K <= 2048 * 2^24 (about 3.4e10); larger returns
+ *     BITNET_ERR_SHAPE.
+ *   - The first call on each device looks up the array's device address
+ *     (with that device current); make that first call before any stream
+ *     capture.
+ *   - All calls share the one array, which keeps the last call's contents;
+ *     every entry a call reads is written earlier in the same call, so
+ *     nothing needs clearing.  Calls that overlap on the GPU (other streams,
+ *     or other threads) race on it: order them on one stream.
+ *   - Non-finite W is not reported (there is no workspace status word). */
+bitnet_status bitnet_quant_weights_noalloc(const float *W, int64_t N, int64_t K, float eps,
+                                           int8_t *Wq, float *gamma, bitnet_stream_t stream);
+
 /* ------------------------------------------------------------------------
  * Failure detection.
  * ------------------------------------------------------------------------ */

@@ -148,6 +148,16 @@ __device__ __forceinline__ int xs_swizzle(int k) {
   return (c << 6) | ((g ^ ((c >> 1) & 3)) << 4) | (k & 15);
 }
 
+// Byte offset of activation k in the block-permuted code row used by the
+// 16-byte streaming GEMV (K % 64 == 0): the 16-byte block g = 4c + e (codes
+// 16g .. 16g + 15) is stored at e * K/4 + 16 c, so the four blocks that meet
+// one 16-byte load of packed weights (64 weights, chunk c) sit K/4 bytes
+// apart and consecutive chunks are consecutive in each quarter.
+__device__ __forceinline__ int xs_blocked(int k, int K) {
+  const int g = k >> 4;
+  return (g & 3) * (K >> 2) + ((g >> 2) << 4) + (k & 15);
+}
+
 // Quantise rows 0..M-1 (M <= MT, K % 16 == 0) of x with one CTA of NT
 // threads.  Pass 1 finds max|t| (and sum x^2 with a gain) per row, keeping
 // up to C 8-element bfloat16 chunks per thread in registers; one
@@ -155,11 +165,13 @@ __device__ __forceinline__ int xs_swizzle(int k) {
 // writes the codes to dst (row stride dst_stride, generic address) and
 // leaves per-warp partial code sums in S.qpart: the caller's next
 // __syncthreads publishes both.  scale[m] is returned to every thread.
+// The group is threads [tid_base, tid_base + NT) of the block.
 template <int NT, int MT, int C, bool SMEM_SRC = false, int BAR = 0, bool SWZ = false>
 __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dtype, int64_t row_bytes, int M,
                                            int K, const float* __restrict__ gain, float rms_eps, int8_t* dst,
-                                           int64_t dst_stride, QuantScratch<NT, MT>& S, float (&scale)[MT]) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+                                           int64_t dst_stride, QuantScratch<NT, MT>& S, float (&scale)[MT],
+                                           int tid_base = 0, bool blocked = false) {
+  const int tid = static_cast<int>(threadIdx.x) - tid_base, lane = tid & 31, warp = tid >> 5;
   const bool cache_ok = (x_dtype == BITNET_BF16);
   uint4 cache[MT][C];
   float am[MT];
@@ -196,6 +208,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
           process(v, k);
         }
       }
+#pragma unroll 4
       for (int k = (C * NT + tid) * 8; k < K; k += NT * 8) {
         uint4 raw[2];
         load8raw<SMEM_SRC>(row, x_dtype, k, raw);
@@ -256,7 +269,8 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
           lo |= (static_cast<uint32_t>(q0) & 0xffu) << (8 * i);
           hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);
         }
-        *reinterpret_cast<uint2*>(drow + (SWZ ? xs_swizzle(k) : k)) = make_uint2(lo, hi);
+        const int off = SWZ ? xs_swizzle(k) : (blocked ? xs_blocked(k, K) : k);
+        *reinterpret_cast<uint2*>(drow + off) = make_uint2(lo, hi);
       };
 #pragma unroll
       for (int c = 0; c < C; ++c) {
@@ -272,6 +286,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
           emit(v, k);
         }
       }
+#pragma unroll 4
       for (int k = (C * NT + tid) * 8; k < K; k += NT * 8) {
         uint4 raw[2];
         load8raw<SMEM_SRC>(row, x_dtype, k, raw);

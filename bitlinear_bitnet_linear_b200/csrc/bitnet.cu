@@ -254,7 +254,7 @@ struct StreamProblem {
 
 template <int MAXP>
 struct StreamPlan {
-  int MT, R, CW, grid, smem;
+  int MT, grid, smem;
   GsParams<MAXP> p;
 };
 
@@ -270,49 +270,56 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
   p.y_dtype = y_dtype;
   p.prequant = prequant ? 1 : 0;
   p.rms_eps = rms_eps;
-  int64_t total = 0, max_rowb = 0, max_rows = 0, Kmax = 0, xmax = 0;
+  int64_t total = 0, max_rowb = 0, Kmax = 0, xmax = 0;
   const int64_t esz = prequant ? 1 : (x_dtype == BITNET_BF16 ? 2 : 4);
   for (int i = 0; i < count; ++i) {
     if (pr[i].K % 64 != 0) return BITNET_ERR_UNSUPPORTED;
     total += pr[i].N * pr[i].K / 4;
     max_rowb = std::max<int64_t>(max_rowb, pr[i].K / 4);
-    max_rows = std::max<int64_t>(max_rows, pr[i].N);
     Kmax = std::max<int64_t>(Kmax, pr[i].K);
     xmax = std::max<int64_t>(xmax, M * pr[i].K * esz);
   }
   p.total_bytes = total;
-  // One CTA per SM.  Large streams get a deep ring; small ones (a single
-  // decode call) a footprint small enough that the next call's CTAs fit
-  // beside them (programmatic dependent launch overlaps their weight streams).
+  // One CTA per SM.  A long stream (many calls in one launch) takes the whole
+  // shared memory for the consumers' rings; a short one (a single decode
+  // call) keeps a footprint that lets the next call's CTAs start beside it.
   const bool big = total >= (int64_t(32) << 20);
   int64_t grid = big ? d->sms : std::min<int64_t>(d->sms, (total + 4095) / 4096);
   if (grid < 1) grid = 1;
   pl.grid = static_cast<int>(grid);
   const int64_t per_cta = (total + grid - 1) / grid;
-  pl.R = pl.MT == 1 ? 4 : (pl.MT == 2 ? 2 : 1);   // largest rows-per-warp task the kernel may pick
-  // eight consumer warps: two rounds of their 10 KB tasks fit in the ring
-  pl.CW = 8;
-  p.deep = big ? 1 : 0;
   p.Kp_max = static_cast<int>(Kmax);
-  const int xs_bytes = pl.MT * p.Kp_max;
-  const int64_t xbuf = (xmax + 127) / 128 * 128;
-  p.nxbuf = (xbuf <= 32 * 1024) ? 2 : 0;
-  p.xbuf_bytes = p.nxbuf ? static_cast<int>(xbuf) : 0;
-  const int budget = big ? d->max_smem_optin : 64 * 1024;
-  int slot = big ? 40 * 1024 : 32 * 1024;
-  if (!big) slot = static_cast<int>(std::min<int64_t>(slot, (per_cta + max_rowb + 15) / 16 * 16));
-  if (slot < max_rowb) slot = static_cast<int>(max_rowb);
-  slot = (slot + 15) / 16 * 16;
-  int room = budget - kGsHeader - xs_bytes - p.nxbuf * p.xbuf_bytes;
-  if (room < slot) room = d->max_smem_optin - kGsHeader - xs_bytes - p.nxbuf * p.xbuf_bytes;
-  int nslots = room / slot;
-  if (nslots > kGsMaxSlots) nslots = kGsMaxSlots;
-  if (!big) nslots = std::min<int64_t>(nslots, std::max<int64_t>(2, (per_cta + slot - 1) / slot + 1));
-  if (nslots < 1) return BITNET_ERR_UNSUPPORTED;
-  p.slot_bytes = slot;
+  // single-token activations are stored block-permuted for the lane-group
+  // tasks; pre-quantised codes are copied as they are (warp tasks)
+  p.blocked = (pl.MT == 1 && !prequant) ? 1 : 0;
+  (void)xmax;
+  // Shapes, most preferred first: (activation buffers, slots per warp, budget).
+  // Two activation buffers let the activation warp run a segment ahead.
+  struct Shape {
+    int nxb, nslots;
+    int64_t budget;
+  };
+  const int64_t small_budget = big ? d->max_smem_optin : 64 * 1024;
+  const Shape shapes[] = {{2, 2, small_budget},
+                          {2, 2, d->max_smem_optin},
+                          {1, 2, d->max_smem_optin},
+                          {2, 1, d->max_smem_optin},
+                          {1, 1, d->max_smem_optin}};
+  int64_t fixed = 0, slot = 0;
+  int nslots = 0;
+  for (const Shape& sh : shapes) {
+    fixed = kGsHeader + sh.nxb * pl.MT * Kmax;
+    slot = (sh.budget - fixed) / (kGsCW * sh.nslots) / 128 * 128;
+    if (slot >= max_rowb) {
+      p.nxb = sh.nxb;
+      nslots = sh.nslots;
+      break;
+    }
+  }
+  if (nslots == 0) return BITNET_ERR_UNSUPPORTED;
+  p.slot_bytes = static_cast<int>(slot);
   p.nslots = nslots;
   int64_t byte0 = 0;
-  const int unit = pl.CW * pl.R;
   for (int i = 0; i < count; ++i) {
     GsProblem& g = p.prob[i];
     g.x = pr[i].x;
@@ -325,39 +332,44 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
     g.K = static_cast<int>(pr[i].K);
     g.N = static_cast<int>(pr[i].N);
     const int64_t rowb = pr[i].K / 4;
-    int64_t sr = slot / rowb;
-    // stage rows aligned to the consumers' task size (16 rows for the 8-lane
-    // group path, 4 for the warp path)
-    const bool lg = pl.MT == 1 && pr[i].K <= 4096 && (pr[i].K / 16) % 8 == 0;
-    const int64_t task = big ? (lg ? 8 : 4) : (lg ? 16 : 4);
-    if (sr >= task) sr -= sr % task;
-    if (big && lg && sr > 8 * pl.CW) sr = 8 * pl.CW;   // one 8-row task per warp per stage
-    (void)unit;
-    g.srows = static_cast<int>(std::max<int64_t>(1, sr));
-    g.pad = 0;
+    int64_t rc = slot / rowb;
+    // a short stream: about one chunk per consumer warp
+    if (!big) rc = std::min<int64_t>(rc, ((per_cta + rowb - 1) / rowb + kGsCW - 1) / kGsCW);
+    rc = std::max<int64_t>(1, std::min<int64_t>(rc, pr[i].N));
+    int task;
+    if (p.blocked) {
+      task = rc >= 8 ? kGsTaskLG2 : kGsTaskLG1;
+      const int64_t unit = task == kGsTaskLG2 ? 8 : 4;
+      if (rc >= unit) rc -= rc % unit;
+    } else {
+      task = kGsTaskWarp;
+      const int64_t unit = pl.MT == 1 ? 4 : (pl.MT == 2 ? 2 : 1);
+      if (rc >= unit) rc -= rc % unit;
+    }
+    g.rc = static_cast<int>(rc);
+    g.task = task;
     g.byte0 = byte0;
     byte0 += pr[i].N * rowb;
   }
-  pl.smem = kGsHeader + xs_bytes + p.nxbuf * p.xbuf_bytes + p.nslots * p.slot_bytes;
+  pl.smem = static_cast<int>(fixed + static_cast<int64_t>(kGsCW) * nslots * slot);
   if (pl.smem > d->max_smem_optin) return BITNET_ERR_UNSUPPORTED;
   return BITNET_OK;
 }
 
-template <int MT, int MAXP, bool DEEP>
+template <int MT, int MAXP>
 cudaError_t run_stream_t(const StreamPlan<MAXP>& pl, cudaStream_t st) {
-  auto k = gemv_stream_kernel<MT, MAXP, 8, DEEP>;
+  auto k = gemv_stream_kernel<MT, MAXP, kGsCW>;
   cudaError_t e = allow_smem(k, pl.smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(k, dim3(pl.grid), dim3(8 * 32 + 32), pl.smem, st, pl.p);
+  return launch_pdl(k, dim3(pl.grid), dim3(kGsCW * 32 + 32), pl.smem, st, pl.p);
 }
 
 template <int MAXP>
 cudaError_t run_stream(const StreamPlan<MAXP>& pl, cudaStream_t st) {
-  const bool deep = pl.p.deep != 0;
   switch (pl.MT) {
-    case 1: return deep ? run_stream_t<1, MAXP, true>(pl, st) : run_stream_t<1, MAXP, false>(pl, st);
-    case 2: return deep ? run_stream_t<2, MAXP, true>(pl, st) : run_stream_t<2, MAXP, false>(pl, st);
-    case 4: return deep ? run_stream_t<4, MAXP, true>(pl, st) : run_stream_t<4, MAXP, false>(pl, st);
+    case 1: return run_stream_t<1, MAXP>(pl, st);
+    case 2: return run_stream_t<2, MAXP>(pl, st);
+    case 4: return run_stream_t<4, MAXP>(pl, st);
     default: return cudaErrorInvalidValue;
   }
 }

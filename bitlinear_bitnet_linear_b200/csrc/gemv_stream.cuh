@@ -11,19 +11,26 @@
 //
 // One launch streams the packed weights of every problem it is given.  The
 // concatenated weight bytes are split evenly over the CTAs; each CTA walks
-// its range as segments (problem, row range).  Roles:
-//   warp 8      producer: cp.async.bulk (TMA, no multicast) of weight stages
-//               into a ring of shared-memory slots and of each segment's raw
-//               activation rows into a small ring, tracked by mbarriers;
-//               weight stages are issued before griddepcontrol.wait (weights
-//               never depend on earlier kernels), activations after it.
-//   warps 0..7  consumers: quantise a segment's activations from shared
-//               memory (fused RMSNorm gain + absmax int8, skipped when the
-//               segment shares the previous one's activations), then
-//               contract every stage's rows, reduce across lanes and write y.
-// Problems that share x (fused Q|K|V, up|gate) are quantised once per CTA.
-// Every wait is bounded: on expiry the kernel records BITNET_ERR_TIMEOUT,
-// stops issuing, lets copies already issued land, and returns.
+// its range as segments (problem, row range), and cuts every segment into
+// chunks of whole rows that fit one shared-memory slot.  Roles:
+//   warps 0..CW-1  consumers.  Chunk j of the CTA belongs to warp j % CW.
+//                  Each consumer keeps its own ring of slots: its lane 0
+//                  issues cp.async.bulk (TMA, no multicast) of its next
+//                  chunks into them, so no consumer ever waits for another
+//                  to release a slot.  The first copies go out before
+//                  griddepcontrol.wait (weights never depend on earlier
+//                  kernels).
+//   warp CW        activations.  Quantises each segment's activations
+//                  (fused RMSNorm gain + absmax int8, skipped when a segment
+//                  shares the previous one's activations) one segment ahead
+//                  of the consumers, into two alternating buffers (one
+//                  when long rows leave no room: then it waits for the
+//                  consumers to finish a segment before quantising the next).
+//                  The first segment is quantised by every warp together.
+// Four warps per scheduler hide the latency of the 128-bit shared loads and
+// of the dp4a chains.  Every wait is bounded: on expiry the kernel records
+// BITNET_ERR_TIMEOUT, stops issuing, lets copies already issued land, and
+// returns.
 #pragma once
 
 #include "act.cuh"
@@ -31,11 +38,16 @@
 
 namespace bitnet {
 
-constexpr int kGsMaxSlots = 12;
-constexpr int kGsMaxX = 2;
+constexpr int kGsMaxS = 4;          // slots per consumer warp
+constexpr int kGsCW = 15;           // consumer warps per CTA
 constexpr int kGsHeader = 2048;
-constexpr int kGsBar = 1;          // named barrier of the consumer warps
-constexpr int kGsPrefetch = 12;    // weight stages pulled into L2 ahead of the ring
+constexpr int kGsBarAll = 1;        // named barrier: every warp of the CTA
+constexpr int kGsBarX = 2;          // named barrier: the activation warp
+
+// Consumer task shapes (per problem).
+constexpr int kGsTaskLG2 = 1;       // M = 1: 8-lane groups, 2 rows each (8-row tasks)
+constexpr int kGsTaskLG1 = 2;       // M = 1: 8-lane groups, 1 row each (4-row tasks)
+constexpr int kGsTaskWarp = 3;      // whole warp over R = 4 / 2 / 1 rows (M = 1 / 2 / 4)
 
 struct GsProblem {
   const void* x;          // [M, K] raw activations (x_dtype) or int8 codes (prequant)
@@ -46,8 +58,8 @@ struct GsProblem {
   void* y;                // [M, N] or nullptr
   int32_t* acc;           // [M, N] exact accumulator export or nullptr
   int K, N;
-  int srows;              // rows per weight stage
-  int pad;
+  int rc;                 // rows per chunk (one slot)
+  int task;               // kGsTask*
   int64_t byte0;          // first byte of this problem in the concatenated weight stream
 };
 
@@ -58,95 +70,121 @@ struct GsParams {
   int M, x_dtype, y_dtype, prequant;
   float rms_eps;
   int64_t total_bytes;
-  int slot_bytes, nslots;        // weight ring
-  int xbuf_bytes, nxbuf;         // activation ring (nxbuf == 0: read x from global memory)
-  int Kp_max;                    // int8 code rows in shared memory, K rounded up to 64
-  int deep;                      // 1: long stream (tasks flow across stages), 0: one short call
+  int slot_bytes, nslots;        // ring of each consumer warp
+  int nxb;                       // activation code buffers (2: quantise a segment ahead)
+  int blocked;                   // 1: codes in the block-permuted layout (lane-group tasks)
+  int Kp_max;                    // int8 code rows in shared memory (K rounded up to 64)
   uint64_t limit_ns;
   uint32_t* status;
 };
 
 template <int MT, int CW>
 struct GsHeader {
-  uint64_t wfull[kGsMaxSlots], wempty[kGsMaxSlots];
-  uint64_t xfull[kGsMaxX], xempty[kGsMaxX];
-  QuantScratch<CW * 32, MT> q;
+  uint64_t wfull[CW][kGsMaxS];
+  uint64_t xfull[2], xfree[2], xcopy;   // xcopy: pre-quantised codes copied in
+  float scale[2][MT];
+  int xsum[2][MT];
+  QuantScratch<(CW + 1) * 32, MT> q;   // first segment (every warp)
+  QuantScratch<32, MT> qx;             // later segments (activation warp)
   int abort;
 };
 
-// First global row (problem, row) of CTA b's share of the weight bytes.
+// First global row (problem, row) of CTA b's share of the weight bytes: the
+// first row that starts at or after byte total * b / gridDim.x (binary
+// search over the problems' byte ranges).
 template <int MAXP>
 __device__ __forceinline__ void gs_cta_start(const GsParams<MAXP>& p, int b, int& prob, int& row) {
   const int64_t target = (p.total_bytes * b) / gridDim.x;
-  for (int i = 0; i < p.nprob; ++i) {
-    const int64_t rb = p.prob[i].K / 4;
-    const int64_t end = p.prob[i].byte0 + rb * p.prob[i].N;
-    if (target < end) {
-      const int64_t r = (target - p.prob[i].byte0 + rb - 1) / rb;
-      if (r < p.prob[i].N) {
-        prob = i;
-        row = static_cast<int>(r);
-        return;
-      }
-    }
+  int lo = 0, hi = p.nprob;   // first problem whose bytes end after target
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    const int64_t end = p.prob[mid].byte0 + static_cast<int64_t>(p.prob[mid].K / 4) * p.prob[mid].N;
+    if (target < end)
+      hi = mid;
+    else
+      lo = mid + 1;
   }
-  prob = p.nprob;
+  prob = lo;
   row = 0;
+  if (lo == p.nprob) return;
+  const int64_t rb = p.prob[lo].K / 4;
+  // target may sit inside the previous problem's last row (before byte0)
+  const int64_t off = target > p.prob[lo].byte0 ? target - p.prob[lo].byte0 : 0;
+  const int64_t r = (off + rb - 1) / rb;
+  if (r < p.prob[lo].N)
+    row = static_cast<int>(r);
+  else
+    prob = lo + 1;            // inside the last row of problem lo: the next one starts at row 0
 }
 
-// Short rows (M = 1, K <= 4096): a warp is four 8-lane groups, each owning
-// RS consecutive rows; a lane walks every eighth code word of its rows, so a
-// row's partial sums are reduced over 8 lanes (3 shuffles).  The groups start
-// their walks 8 words apart (rotation modulo the row length), so rows whose
-// word count is a multiple of 32 do not collide on shared-memory banks.
-// Rows [row0, row0 + 4 RS) of the stage; requires nword % 8 == 0.
+// A chunk position: rows [r, min(r + rc, r1)) of problem q.
+struct GsCursor {
+  int q, r, r1;
+};
+
+// Warp-uniform bounded wait: true only when every lane saw the phase complete.
+__device__ __forceinline__ bool gs_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                        volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, limit_ns, abort_flag));
+}
+
+// M = 1: a warp is four 8-lane groups, each owning RS consecutive rows of
+// the chunk.  A lane reads 16 bytes of packed codes per row at a time (64
+// weights, chunk c = lj, lj + 8, ...) and the four 16-byte activation blocks
+// they meet from the block-permuted code row (xs_blocked), all with 128-bit
+// shared loads; the eight lanes of a group read 128 consecutive bytes, so no
+// load has a bank conflict.  A row's partial sums are reduced over its 8
+// lanes (3 shuffles).  Rows [row0, row0 + 4 RS) of the chunk.
 template <int RS>
-__device__ __forceinline__ void gs_task_lanegroups(const uint32_t* wbase, int rc, int row0, int rowwords, int nword,
-                                                   const int8_t* xs, int lane, int xsum0, float gs0,
-                                                   const GsProblem& P, int r, int y_dtype) {
+__device__ __forceinline__ void gs_task_lg(const uint8_t* wbase, int rc, int row0, int rowb, int nchunk,
+                                           const int8_t* xs, int lane, int xsum0, float gs0, const GsProblem& P,
+                                           int r, int y_dtype) {
   const int lg = lane >> 3, lj = lane & 7;
   const int rb = row0 + lg * RS;                 // this group's first row
   const int nr = max(0, min(RS, rc - rb));
+  const int xq4 = rowb;                          // K / 4: distance between the four block quarters
   int a[RS][4];
 #pragma unroll
   for (int i = 0; i < RS; ++i)
 #pragma unroll
     for (int f = 0; f < 4; ++f) a[i][f] = 0;
-  const uint32_t* wb = wbase + static_cast<int64_t>(rb) * rowwords;
-  int g = lj + 8 * lg;
-  if (g >= nword) g -= nword * (g / nword);
-  if (nr == RS) {
-#pragma unroll 4
-    for (int t = 0; t < nword; t += 8) {
-      uint32_t w[RS];
+  auto body = [&](const uint4 (&w)[RS], const int8_t* xp) {
+    const uint4 xv[4] = {*reinterpret_cast<const uint4*>(xp), *reinterpret_cast<const uint4*>(xp + xq4),
+                         *reinterpret_cast<const uint4*>(xp + 2 * xq4),
+                         *reinterpret_cast<const uint4*>(xp + 3 * xq4)};
 #pragma unroll
-      for (int i = 0; i < RS; ++i) w[i] = wb[i * rowwords + g];
-      const uint4 xv = *reinterpret_cast<const uint4*>(xs + 16 * g);
+    for (int i = 0; i < RS; ++i) {
+      const uint32_t wv[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
 #pragma unroll
-      for (int i = 0; i < RS; ++i) {
-        a[i][0] = dp4a_us(w[i] & 0x03030303u, xv.x, a[i][0]);
-        a[i][1] = dp4a_us(w[i] & 0x0C0C0C0Cu, xv.y, a[i][1]);
-        a[i][2] = dp4a_us(w[i] & 0x30303030u, xv.z, a[i][2]);
-        a[i][3] = dp4a_us(w[i] & 0xC0C0C0C0u, xv.w, a[i][3]);
+      for (int e = 0; e < 4; ++e) {
+        a[i][0] = dp4a_us(wv[e] & 0x03030303u, xv[e].x, a[i][0]);
+        a[i][1] = dp4a_us(wv[e] & 0x0C0C0C0Cu, xv[e].y, a[i][1]);
+        a[i][2] = dp4a_us(wv[e] & 0x30303030u, xv[e].z, a[i][2]);
+        a[i][3] = dp4a_us(wv[e] & 0xC0C0C0C0u, xv[e].w, a[i][3]);
       }
-      g += 8;
-      if (g >= nword) g -= nword;
+    }
+  };
+  const uint8_t* wrow = wbase + static_cast<int64_t>(rb) * rowb + 16 * lj;
+  const int8_t* xp = xs + 16 * lj;
+  if (nr == RS) {
+#pragma unroll 2
+    for (int c = lj; c < nchunk; c += 8) {
+      uint4 w[RS];
+#pragma unroll
+      for (int i = 0; i < RS; ++i) w[i] = *reinterpret_cast<const uint4*>(wrow + i * rowb);
+      body(w, xp);
+      wrow += 128;
+      xp += 128;
     }
   } else if (nr > 0) {
-    for (int t = 0; t < nword; t += 8) {
-      uint32_t w[RS];
+    for (int c = lj; c < nchunk; c += 8) {
+      uint4 w[RS];
 #pragma unroll
-      for (int i = 0; i < RS; ++i) w[i] = (i < nr) ? wb[i * rowwords + g] : 0u;
-      const uint4 xv = *reinterpret_cast<const uint4*>(xs + 16 * g);
-#pragma unroll
-      for (int i = 0; i < RS; ++i) {
-        a[i][0] = dp4a_us(w[i] & 0x03030303u, xv.x, a[i][0]);
-        a[i][1] = dp4a_us(w[i] & 0x0C0C0C0Cu, xv.y, a[i][1]);
-        a[i][2] = dp4a_us(w[i] & 0x30303030u, xv.z, a[i][2]);
-        a[i][3] = dp4a_us(w[i] & 0xC0C0C0C0u, xv.w, a[i][3]);
-      }
-      g += 8;
-      if (g >= nword) g -= nword;
+      for (int i = 0; i < RS; ++i)
+        w[i] = (i < nr) ? *reinterpret_cast<const uint4*>(wrow + i * rowb) : make_uint4(0u, 0u, 0u, 0u);
+      body(w, xp);
+      wrow += 128;
+      xp += 128;
     }
   }
 #pragma unroll
@@ -232,18 +270,16 @@ __device__ __forceinline__ void gs_task_warp(const uint32_t* wbase, int rc, int 
     }
 }
 
-// CW consumer warps + one producer warp.
-template <int MT, int MAXP, int CW, bool DEEP>
-__global__ void __launch_bounds__(CW * 32 + 32, (CW <= 8 ? 2 : 1))
-    gemv_stream_kernel(const __grid_constant__ GsParams<MAXP> p) {
-  constexpr int kGsConsumers = CW * 32;
-  constexpr int kGsWarps = CW;
+// CW consumer warps + one activation warp.
+template <int MT, int MAXP, int CW>
+__global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __grid_constant__ GsParams<MAXP> p) {
+  constexpr int kAll = CW * 32 + 32;
   extern __shared__ __align__(128) uint8_t smem[];
   static_assert(sizeof(GsHeader<MT, CW>) <= kGsHeader, "header too large");
   GsHeader<MT, CW>& H = *reinterpret_cast<GsHeader<MT, CW>*>(smem);
-  int8_t* xs = reinterpret_cast<int8_t*>(smem + kGsHeader);
-  uint8_t* xraw = smem + kGsHeader + MT * p.Kp_max;
-  uint8_t* wring = xraw + p.nxbuf * p.xbuf_bytes;
+  const int xs_stride = MT * p.Kp_max;                       // one activation buffer
+  int8_t* xsbuf = reinterpret_cast<int8_t*>(smem + kGsHeader);
+  uint8_t* wslots = smem + kGsHeader + p.nxb * xs_stride;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int pb, rb, pe, re;
@@ -253,140 +289,185 @@ __global__ void __launch_bounds__(CW * 32 + 32, (CW <= 8 ? 2 : 1))
     pe = p.nprob;
     re = 0;
   }
-  // segment iteration: problem q from pb to pe (inclusive when re > 0)
+  const int qlast = (re > 0) ? pe : pe - 1;
   auto seg_bounds = [&](int q, int& r0, int& r1) {
     r0 = (q == pb) ? rb : 0;
     r1 = (q == pe) ? re : p.prob[q].N;
   };
-  const int qlast = (re > 0) ? pe : pe - 1;
   auto shares_x = [&](int q) {   // segment q reuses segment q-1's quantised activations
     return q > pb && p.prob[q].x == p.prob[q - 1].x && p.prob[q].gain == p.prob[q - 1].gain &&
            p.prob[q].K == p.prob[q - 1].K && p.prob[q].x_scale == p.prob[q - 1].x_scale;
   };
+  // Move a cursor `steps` chunks forward through the CTA's segments.
+  auto advance = [&](GsCursor& c, int steps) {
+    while (c.q <= qlast) {
+      const int rc = p.prob[c.q].rc;
+      if (c.r + steps * rc < c.r1) {   // stays in this segment (the usual case)
+        c.r += steps * rc;
+        return;
+      }
+      steps -= (c.r1 - c.r + rc - 1) / rc;
+      ++c.q;
+      if (c.q <= qlast) seg_bounds(c.q, c.r, c.r1);
+    }
+  };
   const int64_t esz = p.prequant ? 1 : (p.x_dtype == BITNET_BF16 ? 2 : 4);
 
   if (tid == 0) {
-    for (int s = 0; s < p.nslots; ++s) {
-      mbar_init(&H.wfull[s], 1);
-      mbar_init(&H.wempty[s], kGsWarps);
+    for (int w = 0; w < CW; ++w)
+      for (int s = 0; s < p.nslots; ++s) mbar_init(&H.wfull[w][s], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&H.xfull[b], 32);
+      mbar_init(&H.xfree[b], CW);
     }
-    for (int s = 0; s < p.nxbuf; ++s) {
-      mbar_init(&H.xfull[s], 1);
-      mbar_init(&H.xempty[s], kGsWarps);
-    }
+    mbar_init(&H.xcopy, 1);
     H.abort = 0;
     fence_mbar_init();
   }
   __syncthreads();
   volatile int* abort_flag = &H.abort;
 
-  if (warp == kGsWarps) {
-    // ================================================================ producer
-    if (lane != 0) {
-      pdl_launch_dependents();
-      return;
+  GsCursor first{pb, 0, 0};
+  if (pb <= qlast) seg_bounds(pb, first.r, first.r1);
+  advance(first, 0);
+  if (first.q > qlast) {   // empty share (more CTAs than rows)
+    pdl_launch_dependents();
+    return;
+  }
+
+  // ---- consumers: start this warp's weight stream before the dependency wait
+  GsCursor cur = first, icur = first;
+  int issued = 0;
+  uint8_t* myslots = wslots + static_cast<size_t>(warp) * p.nslots * p.slot_bytes;
+  auto issue = [&](int slot) {
+    const GsProblem& Q = p.prob[icur.q];
+    const int64_t rowb = Q.K / 4;
+    const uint32_t bytes = static_cast<uint32_t>(min(Q.rc, icur.r1 - icur.r) * rowb);
+    mbar_expect_tx(&H.wfull[warp][slot], bytes);
+    bulk_g2s(myslots + slot * p.slot_bytes, Q.Wp + static_cast<int64_t>(icur.r) * rowb, bytes, &H.wfull[warp][slot]);
+  };
+  if (warp < CW) {
+    advance(cur, warp);
+    icur = cur;
+    for (int i = 0; i < p.nslots && icur.q <= qlast; ++i) {
+      if (lane == 0) issue(i);
+      advance(icur, CW);
+      ++issued;
     }
-    {
-      int t = 0;          // weight stages issued
-      int u = 0;          // activation buffers issued
-      bool dep_waited = false;
-      bool ok = true;
-      // L2 prefetch cursor: walks the same stage sequence kGsPrefetch stages
-      // ahead of the shared-memory copies, so those copies hit in L2 and the
-      // DRAM stream does not wait for ring slots to be released.
-      int pq = pb, pr = (pb <= qlast) ? rb : 0, npf = 0;
-      auto prefetch_upto = [&](int upto) {
-        while (npf < upto && pq <= qlast) {
-          int q0, q1;
-          seg_bounds(pq, q0, q1);
-          if (pr >= q1) {
-            ++pq;
-            if (pq <= qlast) seg_bounds(pq, pr, q1);
-            continue;
-          }
-          const GsProblem& Q = p.prob[pq];
-          const int64_t qrowb = Q.K / 4;
-          const int rc = min(Q.srows, q1 - pr);
-          bulk_prefetch_l2(Q.Wp + static_cast<int64_t>(pr) * qrowb, static_cast<uint32_t>(rc * qrowb));
-          pr += Q.srows;
-          ++npf;
-        }
-      };
-      prefetch_upto(kGsPrefetch);
-      // Phase 1: fill the weight ring before the dependency wait.
-      {
-        int issued = 0;
-        for (int q = pb; q <= qlast && issued < p.nslots; ++q) {
-          int r0, r1;
-          seg_bounds(q, r0, r1);
-          const GsProblem& P = p.prob[q];
-          const int64_t rowb = P.K / 4;
-          for (int r = r0; r < r1 && issued < p.nslots; r += P.srows) {
-            const int rc = min(P.srows, r1 - r);
-            const uint32_t bytes = static_cast<uint32_t>(rc * rowb);
-            mbar_expect_tx(&H.wfull[issued], bytes);
-            bulk_g2s(wring + issued * p.slot_bytes, P.Wp + static_cast<int64_t>(r) * rowb, bytes, &H.wfull[issued]);
-            ++issued;
-            prefetch_upto(issued + kGsPrefetch);
-          }
-        }
-        t = issued;
-      }
-      // Phase 2: activations (after the dependency wait) and the rest of the weights.
-      int ts = 0;   // global stage index while walking
-      for (int q = pb; q <= qlast && ok; ++q) {
-        int r0, r1;
-        seg_bounds(q, r0, r1);
-        const GsProblem& P = p.prob[q];
-        if (!shares_x(q)) {
-          if (!dep_waited) {
-            pdl_wait();
-            pdl_launch_dependents();
-            dep_waited = true;
-          }
-          if (p.nxbuf > 0) {
-            const int xi = u % p.nxbuf;
-            if (!mbar_wait_bounded(&H.xempty[xi], ((u / p.nxbuf) & 1) ^ 1u, p.limit_ns, abort_flag)) {
-              ok = false;
-              break;
-            }
-            const uint32_t bytes = static_cast<uint32_t>(p.M * P.K * esz);
-            mbar_expect_tx(&H.xfull[xi], bytes);
-            bulk_g2s(xraw + xi * p.xbuf_bytes, P.x, bytes, &H.xfull[xi]);
-          }
-          ++u;
-        }
-        const int64_t rowb = P.K / 4;
-        for (int r = r0; r < r1; r += P.srows, ++ts) {
-          if (ts < t) continue;   // issued in phase 1
-          const int s = ts % p.nslots;
-          if (!mbar_wait_bounded(&H.wempty[s], ((ts / p.nslots) & 1) ^ 1u, p.limit_ns, abort_flag)) {
-            ok = false;
-            break;
-          }
-          const int rc = min(P.srows, r1 - r);
-          const uint32_t bytes = static_cast<uint32_t>(rc * rowb);
-          mbar_expect_tx(&H.wfull[s], bytes);
-          bulk_g2s(wring + s * p.slot_bytes, P.Wp + static_cast<int64_t>(r) * rowb, bytes, &H.wfull[s]);
-          ++t;
-          prefetch_upto(t + kGsPrefetch);
+  }
+  pdl_launch_dependents();
+  pdl_wait();
+
+  // Pre-quantised codes: copy one segment's codes into its buffer and form
+  // their per-row sums (group of NT threads starting at thread tid0).
+  int ncopy = 0;
+  auto copy_codes = [&](const GsProblem& P, int8_t* xs, int Kp, float (&sc)[MT], int* qpart, int nt, int t0,
+                        bool issuer) -> bool {
+    if (issuer) {
+      const uint32_t bytes = static_cast<uint32_t>(p.M * P.K);
+      mbar_expect_tx(&H.xcopy, bytes);
+      bulk_g2s(xs, P.x, bytes, &H.xcopy);
+    }
+    const bool got = gs_wait(&H.xcopy, ncopy & 1, p.limit_ns, abort_flag);
+    if (!got && issuer) mbar_wait_bounded(&H.xcopy, ncopy & 1, p.limit_ns, nullptr);   // let it land
+    ++ncopy;
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      int part = 0;
+      if (got && m < p.M) {
+        for (int k = (tid - t0) * 16; k < P.K; k += nt * 16) {
+          const uint4 v = *reinterpret_cast<const uint4*>(xs + m * Kp + k);
+          part = __dp4a(static_cast<int>(v.x), 0x01010101, part);
+          part = __dp4a(static_cast<int>(v.y), 0x01010101, part);
+          part = __dp4a(static_cast<int>(v.z), 0x01010101, part);
+          part = __dp4a(static_cast<int>(v.w), 0x01010101, part);
         }
       }
-      if (!dep_waited) {
-        pdl_wait();
-        pdl_launch_dependents();
-      }
-      if (!ok) {
-        if (!*abort_flag) {
-          record_error(p.status, BITNET_ERR_TIMEOUT, 0x401u);
-          *abort_flag = 1;
+      part = warp_sum(part);
+      if (lane == 0) qpart[m * (nt / 32) + ((tid - t0) >> 5)] = part;
+      sc[m] = (got && m < p.M) ? __ldg(P.x_scale + m) : 0.0f;
+    }
+    return got;
+  };
+
+  // ---- the first two activation versions, quantised by every warp (the
+  // activation warp then has a whole segment to prepare each later one)
+  bool ok = true;
+  int q1 = pb + 1;                 // segment of version 1
+  while (q1 <= qlast && shares_x(q1)) ++q1;
+  const int ncoop = (q1 <= qlast && p.nxb == 2) ? 2 : 1;
+  for (int cv = 0; cv < ncoop; ++cv) {
+    const GsProblem& P = p.prob[cv == 0 ? pb : q1];
+    int8_t* xs = xsbuf + cv * xs_stride;
+    float sc[MT];
+    const int Kp = (P.K + 63) & ~63;
+    if (p.prequant) {
+      ok = copy_codes(P, xs, Kp, sc, &H.q.qpart[0][0], kAll, 0, tid == CW * 32) && ok;
+    } else {
+      quant_rows<kAll, MT, 1, false, kGsBarAll, false>(static_cast<const char*>(P.x), p.x_dtype, P.K * esz, p.M,
+                                                      P.K, P.gain, p.rms_eps, xs, Kp, H.q, sc, 0, p.blocked != 0);
+    }
+    group_sync<kGsBarAll, kAll>();
+    // the activation warp publishes the version; it reads the shared partials
+    // before any warp can pass the next version's first barrier
+    if (warp == CW) {
+      if (lane == 0) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          int t = 0;
+          for (int w = 0; w < CW + 1; ++w) t += H.q.qpart[m][w];
+          H.xsum[cv][m] = t;
+          H.scale[cv][m] = sc[m];
         }
-        // let every weight copy still in flight land before the CTA exits
-        for (int i = max(0, t - p.nslots); i < t; ++i)
-          mbar_wait_bounded(&H.wfull[i % p.nslots], (i / p.nslots) & 1, p.limit_ns, nullptr);
-        for (int i = max(0, u - p.nxbuf); i < u && p.nxbuf > 0; ++i)
-          mbar_wait_bounded(&H.xfull[i % p.nxbuf], (i / p.nxbuf) & 1, p.limit_ns, nullptr);
       }
+      __syncwarp();
+      mbar_arrive(&H.xfull[cv]);
+    }
+  }
+  if (!ok && tid == 0 && !*abort_flag) {
+    record_error(p.status, BITNET_ERR_TIMEOUT, 0x401u);
+    *abort_flag = 1;
+  }
+
+  if (warp == CW) {
+    // ============================================================ activations
+    int v = ncoop - 1;
+    for (int q = (ncoop == 2 ? q1 : pb) + 1; q <= qlast && ok && !*abort_flag; ++q) {
+      if (shares_x(q)) continue;
+      ++v;
+      const int b = v % p.nxb;
+      if (!gs_wait(&H.xfree[b], ((v / p.nxb) & 1) ^ 1u, p.limit_ns, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const GsProblem& P = p.prob[q];
+      const int Kp = (P.K + 63) & ~63;
+      int8_t* xs = xsbuf + b * xs_stride;
+      float sc[MT];
+      if (p.prequant) {
+        if (!copy_codes(P, xs, Kp, sc, &H.qx.qpart[0][0], 32, CW * 32, lane == 0)) {
+          ok = false;
+          break;
+        }
+      } else {
+        quant_rows<32, MT, 1, false, kGsBarX, false>(static_cast<const char*>(P.x), p.x_dtype, P.K * esz, p.M,
+                                                     P.K, P.gain, p.rms_eps, xs, Kp, H.qx, sc, CW * 32,
+                                                     p.blocked != 0);
+      }
+      __syncwarp();
+      if (lane == 0) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          H.xsum[b][m] = H.qx.qpart[m][0];
+          H.scale[b][m] = sc[m];
+        }
+      }
+      __syncwarp();
+      mbar_arrive(&H.xfull[b]);
+    }
+    if (!ok && lane == 0 && !*abort_flag) {
+      record_error(p.status, BITNET_ERR_TIMEOUT, 0x402u);
+      *abort_flag = 1;
     }
     return;
   }
@@ -394,168 +475,84 @@ __global__ void __launch_bounds__(CW * 32 + 32, (CW <= 8 ? 2 : 1))
   // ================================================================== consumers
   float sc[MT];
   int xsum[MT];
-#pragma unroll
-  for (int m = 0; m < MT; ++m) {
-    sc[m] = 0.0f;
-    xsum[m] = 0;
-  }
-  int ts = 0, u = 0;
-  int64_t task0 = 0;
-  bool triggered = false;
-  for (int q = pb; q <= qlast; ++q) {
-    int r0, r1;
-    seg_bounds(q, r0, r1);
-    const GsProblem& P = p.prob[q];
-    const int Kp = (P.K + 63) & ~63;
-    if (!shares_x(q)) {
-      // all consumers are done with the previous segment's codes
-      group_sync<kGsBar, kGsConsumers>();
-      bool have = true;
-      const char* src = static_cast<const char*>(P.x);
-      if (p.nxbuf > 0) {
-        const int xi = u % p.nxbuf;
-        have = mbar_wait_bounded(&H.xfull[xi], (u / p.nxbuf) & 1, p.limit_ns, abort_flag);
-        src = reinterpret_cast<const char*>(xraw + xi * p.xbuf_bytes);
-      } else {
-        pdl_wait();
+  int v = -1, t = 0, slot = 0;
+  uint32_t phase = 0;
+  float gamma_next = 0.0f;
+  for (int q = pb; q <= qlast && ok; ++q) {
+    if (q == pb || !shares_x(q)) {
+      if (v >= 0) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&H.xfree[v % p.nxb]);
       }
-      if (!have && !*abort_flag) {
-        record_error(p.status, BITNET_ERR_TIMEOUT, 0x402u);
-        *abort_flag = 1;
+      ++v;
+      if (!gs_wait(&H.xfull[v % p.nxb], (v / p.nxb) & 1, p.limit_ns, abort_flag)) {
+        ok = false;
+        break;
       }
-      const bool live = !*abort_flag;
-      if (p.prequant) {
-        // copy codes (swizzled) and form their sums
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          int part = 0;
-          if (live && m < p.M) {
-            for (int k = tid * 16; k < P.K; k += kGsConsumers * 16) {
-              const uint4 v = p.nxbuf > 0 ? *reinterpret_cast<const uint4*>(src + m * P.K + k)
-                                          : __ldg(reinterpret_cast<const uint4*>(src + m * P.K + k));
-              *reinterpret_cast<uint4*>(xs + m * Kp + k) = v;
-              part = __dp4a(static_cast<int>(v.x), 0x01010101, part);
-              part = __dp4a(static_cast<int>(v.y), 0x01010101, part);
-              part = __dp4a(static_cast<int>(v.z), 0x01010101, part);
-              part = __dp4a(static_cast<int>(v.w), 0x01010101, part);
-            }
-          }
-          part = warp_sum(part);
-          if (lane == 0) H.q.qpart[m][warp] = part;
-          sc[m] = (live && m < p.M) ? __ldg(P.x_scale + m) : 0.0f;
-        }
-      } else if (live) {
-        if (p.nxbuf > 0)
-          quant_rows<kGsConsumers, MT, (MT == 1 ? 2 : 1), true, kGsBar, false>(
-              src, p.x_dtype, P.K * esz, p.M, P.K, P.gain, p.rms_eps, xs, Kp, H.q, sc);
-        else
-          quant_rows<kGsConsumers, MT, (MT == 1 ? 2 : 1), false, kGsBar, false>(
-              src, p.x_dtype, P.K * esz, p.M, P.K, P.gain, p.rms_eps, xs, Kp, H.q, sc);
-      } else {
-        group_sync<kGsBar, kGsConsumers>();   // the barrier inside quant_rows
-      }
-      // zero padding: codes past K (within the last 64-wide chunk) and rows past M
-      for (int m = 0; m < MT; ++m) {
-        const int k0 = (m < p.M) ? P.K : 0;
-        for (int k = k0 + tid * 16; k < Kp; k += kGsConsumers * 16)
-          *reinterpret_cast<uint4*>(xs + m * Kp + k) = make_uint4(0, 0, 0, 0);
-      }
-      group_sync<kGsBar, kGsConsumers>();
-      if (p.nxbuf > 0 && lane == 0) mbar_arrive(&H.xempty[u % p.nxbuf]);
-      ++u;
 #pragma unroll
       for (int m = 0; m < MT; ++m) {
-        int t = 0;
-#pragma unroll
-        for (int w = 0; w < kGsWarps; ++w) t += H.q.qpart[m][w];
-        xsum[m] = t;
-      }
-      if (!triggered) {
-        pdl_launch_dependents();
-        triggered = true;
+        sc[m] = H.scale[v % p.nxb][m];
+        xsum[m] = H.xsum[v % p.nxb][m];
       }
     }
-
-    const float gamma = __ldg(P.gamma);
-    const int64_t rowb = P.K / 4;
-    const int nword = P.K / 16;      // 32-bit code words (16 weights) per row
-    const int rowwords = static_cast<int>(rowb / 4);
-    // Work units ("tasks") of every stage are numbered globally and dealt to
-    // the warps round-robin, so a warp with nothing to do in one stage moves
-    // on to the next; a slot is released when every warp has passed it.
-    const bool lanegroups = (MT == 1) && (P.K <= 4096) && (nword % 8 == 0);
+    const GsProblem& P = p.prob[q];
+    const int8_t* xs = xsbuf + (v % p.nxb) * xs_stride;
+    const int Kp = (P.K + 63) & ~63;
+    const float gamma = (q == pb) ? __ldg(P.gamma) : gamma_next;
+    if (q < qlast) gamma_next = __ldg(p.prob[q + 1].gamma);   // in flight during this segment
     const float gs0 = __fmul_rn(gamma, sc[0]);
-    for (int r = r0; r < r1; r += P.srows, ++ts) {
-      const int s = ts % p.nslots;
-      const int rc = min(P.srows, r1 - r);
-      // task size for this stage (identical in every warp): the largest that
-      // still gives every warp work, up to 16 rows (4 per 8-lane group) or 4
-      // rows per warp
-      int kind, rows_per_task;
-      if constexpr (DEEP) {
-        // long streams: fixed task sizes (8-row lane-group tasks; 4/2/1-row
-        // warp tasks by M); stages hold one task per warp
-        kind = lanegroups ? 2 : (MT == 1 ? 4 : (MT == 2 ? 2 : 1));
-        rows_per_task = lanegroups ? 4 * kind : kind;
-      } else if (lanegroups) {
-        kind = ((rc + 15) / 16 >= kGsWarps) ? 4 : 1;
-        rows_per_task = 4 * kind;
-      } else {
-        auto cost = [&](int RR) { return ((rc + RR - 1) / RR + kGsWarps - 1) / kGsWarps * RR; };
-        kind = 1;
-        if (MT <= 2 && cost(2) <= cost(1)) kind = 2;
-        if (MT == 1 && cost(4) <= cost(kind)) kind = 4;
-        rows_per_task = kind;
+    const int nword = P.K / 16;      // 32-bit code words (16 weights) per row
+    const int rowb = P.K / 4, nchunk = P.K / 64;
+    while (cur.q == q) {
+      if (!gs_wait(&H.wfull[warp][slot], phase, p.limit_ns, abort_flag)) {
+        ok = false;
+        break;
       }
-      const int nt = (rc + rows_per_task - 1) / rows_per_task;
-      const int j0 = (warp - static_cast<int>(task0 % kGsWarps) + kGsWarps) % kGsWarps;
-      // Every warp waits for every stage to land, even one with no task in
-      // it, before releasing it: a warp is then never more than one phase of
-      // a slot ahead of the others, which keeps the parity waits and the
-      // release counts of each slot's barriers exact.
-      const bool got = mbar_wait_bounded(&H.wfull[s], (ts / p.nslots) & 1, p.limit_ns, abort_flag);
-      if (!got && !*abort_flag) {
+      const uint8_t* wb8 = myslots + slot * p.slot_bytes;
+      const int rows = min(P.rc, cur.r1 - cur.r);
+      const int r = cur.r;
+      if (MT == 1 && P.task == kGsTaskLG2) {
+        for (int row0 = 0; row0 < rows; row0 += 8)
+          gs_task_lg<2>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+      } else if (MT == 1 && P.task == kGsTaskLG1) {
+        for (int row0 = 0; row0 < rows; row0 += 4)
+          gs_task_lg<1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+      } else {
+        constexpr int R = (MT == 1) ? 4 : ((MT == 2) ? 2 : 1);
+        const uint32_t* wbase = reinterpret_cast<const uint32_t*>(wb8);
+        for (int row0 = 0; row0 < rows; row0 += R)
+          gs_task_warp<R, MT>(wbase, rows, row0, nword, nword, xs, Kp, lane, xsum, sc, gamma, P, r, p.M,
+                              p.y_dtype);
+      }
+      __syncwarp();
+      if (icur.q <= qlast) {
+        if (lane == 0) {
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          issue(slot);
+        }
+        advance(icur, CW);
+        ++issued;
+      }
+      advance(cur, CW);
+      ++t;
+      if (++slot == p.nslots) {
+        slot = 0;
+        phase ^= 1u;
+      }
+    }
+  }
+  if (!ok) {
+    if (lane == 0) {
+      if (!*abort_flag) {
         record_error(p.status, BITNET_ERR_TIMEOUT, 0x403u);
         *abort_flag = 1;
       }
-      if (j0 < nt) {
-        if (got) {
-          const uint32_t* wbase = reinterpret_cast<const uint32_t*>(wring + s * p.slot_bytes);
-          for (int j = j0; j < nt; j += kGsWarps) {
-            const int row0 = j * rows_per_task;
-            if (lanegroups) {
-              if constexpr (DEEP) {
-                gs_task_lanegroups<2>(wbase, rc, row0, rowwords, nword, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
-              } else {
-                if (kind == 4)
-                  gs_task_lanegroups<4>(wbase, rc, row0, rowwords, nword, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
-                else
-                  gs_task_lanegroups<1>(wbase, rc, row0, rowwords, nword, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
-              }
-            } else if constexpr (DEEP) {
-              gs_task_warp<(MT == 1 ? 4 : (MT == 2 ? 2 : 1)), MT>(wbase, rc, row0, rowwords, nword, xs, Kp, lane, xsum,
-                                                                   sc, gamma, P, r, p.M, p.y_dtype);
-            } else if (kind == 4) {
-              if constexpr (MT == 1)
-                gs_task_warp<4, MT>(wbase, rc, row0, rowwords, nword, xs, Kp, lane, xsum, sc, gamma, P, r, p.M,
-                                    p.y_dtype);
-            } else if (kind == 2) {
-              if constexpr (MT <= 2)
-                gs_task_warp<2, MT>(wbase, rc, row0, rowwords, nword, xs, Kp, lane, xsum, sc, gamma, P, r, p.M,
-                                    p.y_dtype);
-            } else {
-              gs_task_warp<1, MT>(wbase, rc, row0, rowwords, nword, xs, Kp, lane, xsum, sc, gamma, P, r, p.M,
-                                  p.y_dtype);
-            }
-          }
-        }
-      }
-      task0 += nt;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&H.wempty[s]);
+      // let this warp's weight copies still in flight land before the CTA exits
+      for (int i = t; i < issued; ++i)
+        mbar_wait_bounded(&H.wfull[warp][i % p.nslots], (i / p.nslots) & 1, p.limit_ns, nullptr);
     }
+    __syncwarp();
   }
-  if (!triggered) pdl_launch_dependents();
 }
 
 }  // namespace bitnet

@@ -338,9 +338,10 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
     rc = std::max<int64_t>(1, std::min<int64_t>(rc, pr[i].N));
     int task;
     if (p.blocked) {
-      task = rc >= 8 ? kGsTaskLG2 : kGsTaskLG1;
-      const int64_t unit = task == kGsTaskLG2 ? 8 : 4;
-      if (rc >= unit) rc -= rc % unit;
+      // the largest lane-group task whose rows fit the chunk
+      task = rc >= 8 ? kGsTaskG8R2 : (rc >= 4 ? kGsTaskG16R2 : (rc >= 2 ? kGsTaskG16R1 : kGsTaskG32R1));
+      const int64_t unit = task == kGsTaskG8R2 ? 8 : (task == kGsTaskG16R2 ? 4 : (task == kGsTaskG16R1 ? 2 : 1));
+      rc -= rc % unit;
     } else {
       task = kGsTaskWarp;
       const int64_t unit = pl.MT == 1 ? 4 : (pl.MT == 2 ? 2 : 1);
@@ -399,13 +400,38 @@ cudaError_t run_tc_t(const int8_t* xq, const TcParams& p, cudaStream_t st) {
   return launch_pdl(k, grid, dim3(kTcThreads), smem, st, map, p);
 }
 
-// Token tile BM = MMA N.  With 4 TMEM A buffers every configuration holds at
-// most 256 TMEM columns, so two CTAs can share an SM.
-cudaError_t run_tc(const int8_t* xq, const TcParams& p, cudaStream_t st) {
+// Persistent tiles of 256 weight rows x BM tokens, one CTA per SM (the
+// shared-memory request keeps a second CTA off the SM: both want all 512
+// TMEM columns).
+template <int BM, int SS, int AS>
+cudaError_t run_tp_t(const int8_t* xq, const TcParams& p, int sms, cudaStream_t st) {
+  static_assert(2 * tp_smem_bytes<BM, SS, AS>() > 233472, "one CTA per SM");
+  CUtensorMap map;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.K), static_cast<cuuint64_t>(p.M)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.K)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcBK), static_cast<cuuint32_t>(BM)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<int8_t*>(xq), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  auto k = tc_gemm_persistent_kernel<BM, SS, AS>;
+  constexpr int smem = tp_smem_bytes<BM, SS, AS>();
+  cudaError_t e = allow_smem(k, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = static_cast<int64_t>((p.N + kTpRows - 1) / kTpRows) * ((p.M + BM - 1) / BM);
+  const int grid = static_cast<int>(std::min<int64_t>(tiles, sms));
+  return launch_pdl(k, dim3(grid), dim3(kTpThreads), smem, st, map, p);
+}
+
+// Token tile BM = MMA N.  Up to 64 tokens: one CTA per 128-row tile, 4 TMEM
+// A buffers, at most 256 TMEM columns, so two CTAs can share an SM.  Beyond:
+// the persistent kernel.
+cudaError_t run_tc(const int8_t* xq, const TcParams& p, int sms, cudaStream_t st) {
   if (p.M <= 16) return run_tc_t<16, 8, 4>(xq, p, st);
   if (p.M <= 32) return run_tc_t<32, 8, 4>(xq, p, st);
   if (p.M <= 64) return run_tc_t<64, 8, 4>(xq, p, st);
-  return run_tc_t<128, 6, 4>(xq, p, st);
+  return run_tp_t<128, 6, 4>(xq, p, sms, st);
 }
 
 bitnet_status launch_result(cudaError_t e) {
@@ -679,7 +705,7 @@ static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in
   p.wvec = (K % 64 == 0) ? 1 : 0;
   p.limit_ns = limit;
   p.status = status;
-  return launch_result(run_tc(xq, p, st));
+  return launch_result(run_tc(xq, p, d->sms, st));
 }
 
 bitnet_status bitnet_linear_ex(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t* Wp, int64_t N,

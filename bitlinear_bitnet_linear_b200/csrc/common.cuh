@@ -191,6 +191,17 @@ __device__ __forceinline__ void tc_mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, u
       : "memory");
 }
 
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::i8, one CTA.
+__device__ __forceinline__ void tc_mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
                : "memory");
@@ -268,6 +279,20 @@ __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   return v;
+}
+
+// Exact int -> binary32 for |a| < 2^22 on the integer pipes: 1.5 * 2^23 has
+// a unit in the last place of 1, so its bit pattern plus a is the binary32
+// of 1.5 * 2^23 + a, and subtracting 1.5 * 2^23 is exact.
+__device__ __forceinline__ float small_int_to_float(int a) {
+  return __fsub_rn(__int_as_float(0x4B400000 + a), 12582912.0f);
+}
+
+// binary32 -> bfloat16 bits, round to nearest, ties to even, for finite
+// values: add 0x7FFF plus the lowest kept bit, keep the top 16 bits.
+__device__ __forceinline__ uint16_t bf16_bits_rne(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return static_cast<uint16_t>((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
 }
 
 __device__ __forceinline__ void store_y(void* y, int y_dtype, int64_t idx, float v) {

@@ -290,6 +290,318 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Persistent variant (M > 64): one CTA per SM walks output tiles of 256
+// weight rows x BM tokens.  Each 128-wide K block feeds two M = 128 MMAs (the
+// two weight-row halves) that share one activation stage, halving the L2
+// traffic per MAC of a 128-row tile.  Both operands come from shared memory:
+// the converters expand the 2-bit codes to one unsigned byte per weight and
+// store them, 16 bytes at a time, in the 128-byte-swizzled K-major layout
+// that the TMA gives the activations.  All 512 TMEM columns hold two
+// accumulator buffers (2 x 2 halves x BM columns), so the epilogue of tile i
+// runs while the MMAs of tile i + 1 fill the other buffer.
+// Roles (576 threads):
+//   warp 0        TMA producer, running ahead across tiles (SS stages)
+//   warp 1        TMEM allocator and single-thread MMA issuer
+//   warps 2..9    converters: one weight row per thread (AS stages)
+//   warps 10..17  epilogue: one weight row per thread (half (w-10)/4, TMEM
+//                 lane quadrant w % 4)
+// Pipeline waits suspend in hardware (try_wait with a time hint), so warps
+// with nothing to do take no issue slots from the others; only the MMA
+// issuer, on the critical path, spins on its operand barriers.
+// Barriers: full/sempty (activation stages), afull/aempty (A stages; 256
+// converter arrivals), dfull[b] (all MMAs of a tile done), dfree[b] (8
+// epilogue warps done reading buffer b), mdone (every MMA issued has
+// completed, before TMEM is freed).
+// ---------------------------------------------------------------------------
+constexpr int kTpRows = 256;
+constexpr int kTpThreads = 18 * 32;
+constexpr int kTpAStage = kTpRows * kTcBK;     // 32 KB of expanded codes per K block
+
+template <int BM, int SS, int AS>
+__host__ __device__ constexpr int tp_smem_bytes() {
+  return 1024 /* alignment slack */ + SS * BM * kTcBK + AS * kTpAStage + 1024 /* barriers, flags */;
+}
+
+template <int BM, int SS, int AS>
+__global__ void __launch_bounds__(kTpThreads, 1)
+    tc_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
+  static_assert(BM == 128, "two buffers of 2 x BM accumulator columns fill TMEM");
+  constexpr uint32_t kCols = 512;
+  constexpr uint32_t kStageBytes = BM * kTcBK;
+  constexpr uint32_t kIdesc = idesc_i8_us(kTcBN, BM);
+  constexpr int kPD = 4;                               // converter prefetch depth (K blocks)
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* xs = smem;
+  uint8_t* as = smem + SS * kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(as + AS * kTpAStage);
+  uint64_t* sempty = full + SS;
+  uint64_t* afull = sempty + SS;
+  uint64_t* aempty = afull + AS;
+  uint64_t* dfull = aempty + AS;
+  uint64_t* dfree = dfull + 2;
+  uint64_t* mdone = dfree + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mdone + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int KB = p.KB;
+  const int n_tiles = (p.N + kTpRows - 1) / kTpRows;
+  const int tiles = n_tiles * ((p.M + BM - 1) / BM);
+  const int G = gridDim.x;
+  // local tile i of this CTA: global tile blockIdx.x + i * G; tiles of one
+  // token block are adjacent, so CTAs running together share activation tiles
+  const int my_tiles = blockIdx.x < tiles ? (tiles - 1 - blockIdx.x) / G + 1 : 0;
+  auto tile_m0 = [&](int i) { return ((blockIdx.x + i * G) / n_tiles) * BM; };
+  auto tile_n0 = [&](int i) { return ((blockIdx.x + i * G) % n_tiles) * kTpRows; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < SS; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&sempty[s], 1);
+    }
+    for (int a = 0; a < AS; ++a) {
+      mbar_init(&afull[a], 256);
+      mbar_init(&aempty[a], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&dfull[b], 1);
+      mbar_init(&dfree[b], 8);
+    }
+    mbar_init(mdone, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) prefetch_tensormap(&tmap_x);
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, kCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+
+  auto fail = [&](uint32_t site) {
+    record_error(p.status, BITNET_ERR_TIMEOUT, site);
+    *abort_flag = 1;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      pdl_wait();   // activations come from the previous kernel
+      int g = 0;
+      bool ok = true;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const int m0 = tile_m0(i);
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          const int s = g % SS;
+          if (!mbar_wait_sleep(&sempty[s], ((g / SS) & 1) ^ 1u, p.limit_ns, abort_flag)) {
+            if (!*abort_flag) fail(0x311u);
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[s], kStageBytes);
+          tma_load_2d(xs + s * kStageBytes, &tmap_x, kb * kTcBK, m0, &full[s]);
+        }
+      }
+      if (!ok) {
+        // let every copy already issued land before the CTA can exit
+        for (int j = max(0, g - SS); j < g; ++j) mbar_wait_bounded(&full[j % SS], (j / SS) & 1, p.limit_ns, nullptr);
+      }
+    }
+    pdl_launch_dependents();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      int g = 0;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const int b = i & 1;
+        // the epilogue has read what the tile before last left in buffer b
+        if (!mbar_wait_sleep(&dfree[b], ((i >> 1) & 1) ^ 1u, p.limit_ns, abort_flag)) {
+          if (!*abort_flag) fail(0x312u);
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d0 = tmem + static_cast<uint32_t>(b * 2 * BM);
+        for (int kb = 0; kb < KB; ++kb, ++g) {
+          const int s = g % SS;
+          const int a = g % AS;
+          // the issuer is the critical path: it spins (one thread), the others sleep
+          if (!mbar_wait_bounded(&full[s], (g / SS) & 1, p.limit_ns, abort_flag) ||
+              !mbar_wait_bounded(&afull[a], (g / AS) & 1, p.limit_ns, abort_flag)) {
+            if (!*abort_flag) fail(0x313u);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xs + s * kStageBytes));
+          const uint64_t adesc0 = smem_desc_k_sw128(smem_u32(as + a * kTpAStage));
+          const uint64_t adesc1 = smem_desc_k_sw128(smem_u32(as + a * kTpAStage + kTpAStage / 2));
+#pragma unroll
+          for (int j = 0; j < kTcBK / 32; ++j) {
+            // K step of 32 bytes: advance both descriptors' start address by 32 B (>> 4 = 2)
+            const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
+            tc_mma_i8_ss(d0, adesc0 + 2ull * j, bdesc + 2ull * j, kIdesc, acc);
+            tc_mma_i8_ss(d0 + BM, adesc1 + 2ull * j, bdesc + 2ull * j, kIdesc, acc);
+          }
+          tc_commit(&sempty[s]);
+          tc_commit(&aempty[a]);
+        }
+        if (ok) tc_commit(&dfull[b]);
+      }
+      // every MMA issued has completed before TMEM can be freed
+      tc_commit(mdone);
+      mbar_wait_bounded(mdone, 0, p.limit_ns, nullptr);
+    }
+    pdl_launch_dependents();
+  } else if (warp < 10) {
+    // ------------------------------------------------------------ converters
+    const int row = (warp - 2) * 32 + lane;          // A row of the 256-row tile
+    const int rowbytes = p.K / 4;
+    const int total = my_tiles * KB;
+    uint32_t wb[kPD][8];
+    auto load = [&](int gi, uint32_t (&w)[8]) {
+      const int i = gi / KB, kb = gi - i * KB;
+      const int n = tile_n0(i) + row;
+      const bool valid = n < p.N;
+      tc_load_row_block(p.Wp + static_cast<int64_t>(valid ? n : 0) * rowbytes, valid, rowbytes, kb, p.wvec, w);
+    };
+#pragma unroll
+    for (int j = 0; j < kPD; ++j)
+      if (j < total) load(j, wb[j]);
+    // 16-byte chunk c of this row sits at chunk c ^ (row % 8) (128-byte swizzle)
+    const uint32_t swz = static_cast<uint32_t>(row & 7);
+    bool ok = true;
+    for (int g0 = 0; g0 < total && ok; g0 += kPD) {
+#pragma unroll
+      for (int j = 0; j < kPD; ++j) {
+        const int g = g0 + j;
+        if (g < total && ok) {
+          const int a = g % AS;
+          if (!mbar_wait_sleep(&aempty[a], ((g / AS) & 1) ^ 1u, p.limit_ns, abort_flag)) {
+            if (!*abort_flag) fail(0x314u);
+            ok = false;
+          } else {
+            uint8_t* arow = as + a * kTpAStage + row * kTcBK;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              // word c covers weights 16c .. 16c + 15: field s holds 16c + 4s .. + 3
+              const uint32_t w = wb[j][c];
+              *reinterpret_cast<uint4*>(arow + ((static_cast<uint32_t>(c) ^ swz) << 4)) =
+                  make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u, (w >> 4) & 0x03030303u,
+                             (w >> 6) & 0x03030303u);
+            }
+            // the tensor core reads these bytes through the async proxy
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            mbar_arrive(&afull[a]);
+            if (g + kPD < total) load(g + kPD, wb[j]);
+          }
+        }
+      }
+    }
+    pdl_launch_dependents();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int h = (warp - 10) >> 2;
+    const int q = warp & 3;
+    const int row = h * 128 + q * 32 + lane;
+    const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    constexpr int kChunks = BM / 32;
+    const bool fast = p.y != nullptr && p.acc == nullptr && p.y_dtype == BITNET_BF16 && p.K <= 32768;
+    pdl_wait();   // token scales and sums come from the previous kernel
+    const float gamma = __ldg(p.gamma);
+    const float* __restrict__ xsc = p.x_scale;
+    const int32_t* __restrict__ xsm = p.x_sum;
+    for (int i = 0; i < my_tiles; ++i) {
+      const int b = i & 1;
+      const int m0 = tile_m0(i);
+      const int n = tile_n0(i) + row;
+      const bool valid = n < p.N;
+      // lane l holds token (m0 + 32 c + l)'s scale and code sum: loaded before
+      // the accumulators are ready, shuffled out below
+      float gs[kChunks];
+      int xsum[kChunks];
+#pragma unroll
+      for (int c = 0; c < kChunks; ++c) {
+        const int mi = m0 + 32 * c + lane;
+        gs[c] = 0.0f;
+        xsum[c] = 0;
+        if (mi < p.M) {
+          gs[c] = __fmul_rn(gamma, __ldg(xsc + mi));
+          xsum[c] = __ldg(xsm + mi);
+        }
+      }
+      const bool got = mbar_wait_sleep(&dfull[b], (i >> 1) & 1, p.limit_ns, abort_flag);
+      if (!got && !*abort_flag) fail(0x315u);
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      if (i + 1 == my_tiles) pdl_launch_dependents();
+      const uint32_t dcol = static_cast<uint32_t>(b * 2 * BM + h * BM);
+      // A rolled loop over the 32-token chunks keeps the (unrolled) chunk
+      // body in the instruction cache: fully unrolled, the epilogue is
+      // straight-line code that runs once per tile and misses on every fetch.
+#pragma unroll 1
+      for (int c = 0; c < kChunks; ++c) {
+        if (m0 + 32 * c >= p.M) break;   // warp-uniform
+        float gsc = gs[0];
+        int xsc_ = xsum[0];
+#pragma unroll
+        for (int u = 1; u < kChunks; ++u)
+          if (c == u) {
+            gsc = gs[u];
+            xsc_ = xsum[u];
+          }
+        uint32_t v[32];
+        tmem_ld_32x32b_x32(tmem + lane_base + dcol + static_cast<uint32_t>(32 * c), v);
+        tc_wait_ld();
+        if (fast) {
+          // |acc| <= 128 K <= 2^22: conversions on the integer pipes (the
+          // conversion unit would otherwise bound the epilogue)
+          uint16_t* yb = static_cast<uint16_t*>(p.y) + static_cast<int64_t>(m0 + 32 * c) * p.N + n;
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const float gst = __shfl_sync(0xffffffffu, gsc, t);
+            const int xst = __shfl_sync(0xffffffffu, xsc_, t);
+            if (valid && m0 + 32 * c + t < p.M)
+              yb[static_cast<int64_t>(t) * p.N] =
+                  bf16_bits_rne(__fmul_rn(small_int_to_float(static_cast<int>(v[t]) - xst), gst));
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const float gst = __shfl_sync(0xffffffffu, gsc, t);
+            const int xst = __shfl_sync(0xffffffffu, xsc_, t);
+            const int m = m0 + 32 * c + t;
+            if (valid && m < p.M) {
+              const int acc = static_cast<int>(v[t]) - xst;
+              const int64_t idx = static_cast<int64_t>(m) * p.N + n;
+              if (p.acc != nullptr) p.acc[idx] = acc;
+              if (p.y != nullptr) store_y(p.y, p.y_dtype, idx, __fmul_rn(__int2float_rn(acc), gst));
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&dfree[b]);
+    }
+    pdl_launch_dependents();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kCols);
+  }
+}
+
 // Watchdog self-test: wait on a barrier that nothing completes.
 __global__ void watchdog_selftest_kernel(uint64_t limit_ns, uint32_t* status) {
   __shared__ uint64_t bar;

@@ -44,10 +44,13 @@ constexpr int kGsHeader = 2048;
 constexpr int kGsBarAll = 1;        // named barrier: every warp of the CTA
 constexpr int kGsBarX = 2;          // named barrier: the activation warp
 
-// Consumer task shapes (per problem).
-constexpr int kGsTaskLG2 = 1;       // M = 1: 8-lane groups, 2 rows each (8-row tasks)
-constexpr int kGsTaskLG1 = 2;       // M = 1: 8-lane groups, 1 row each (4-row tasks)
-constexpr int kGsTaskWarp = 3;      // whole warp over R = 4 / 2 / 1 rows (M = 1 / 2 / 4)
+// Consumer task shapes (per problem): lane groups of G lanes with RS rows
+// each (M = 1, block-permuted codes), or whole warps.
+constexpr int kGsTaskG8R2 = 0;      // 8-row tasks
+constexpr int kGsTaskG16R2 = 1;     // 4-row tasks
+constexpr int kGsTaskG16R1 = 2;     // 2-row tasks
+constexpr int kGsTaskG32R1 = 3;     // 1-row tasks
+constexpr int kGsTaskWarp = 4;      // whole warp over R = 4 / 2 / 1 rows (M = 1 / 2 / 4), linear codes
 
 struct GsProblem {
   const void* x;          // [M, K] raw activations (x_dtype) or int8 codes (prequant)
@@ -128,18 +131,18 @@ __device__ __forceinline__ bool gs_wait(uint64_t* bar, uint32_t parity, uint64_t
   return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, limit_ns, abort_flag));
 }
 
-// M = 1: a warp is four 8-lane groups, each owning RS consecutive rows of
-// the chunk.  A lane reads 16 bytes of packed codes per row at a time (64
-// weights, chunk c = lj, lj + 8, ...) and the four 16-byte activation blocks
-// they meet from the block-permuted code row (xs_blocked), all with 128-bit
-// shared loads; the eight lanes of a group read 128 consecutive bytes, so no
-// load has a bank conflict.  A row's partial sums are reduced over its 8
-// lanes (3 shuffles).  Rows [row0, row0 + 4 RS) of the chunk.
-template <int RS>
+// M = 1: a warp is 32/G groups of G lanes (G = 8, 16 or 32), each owning RS
+// consecutive rows of the chunk.  A lane reads 16 bytes of packed codes per
+// row at a time (64 weights, chunk c = lj, lj + G, ...) and the four 16-byte
+// activation blocks they meet from the block-permuted code row (xs_blocked),
+// all with 128-bit shared loads; every 8 consecutive lanes read 128
+// consecutive bytes, so no load has a bank conflict.  A row's partial sums
+// are reduced over its G lanes.  Rows [row0, row0 + (32/G) RS) of the chunk.
+template <int G, int RS>
 __device__ __forceinline__ void gs_task_lg(const uint8_t* wbase, int rc, int row0, int rowb, int nchunk,
                                            const int8_t* xs, int lane, int xsum0, float gs0, const GsProblem& P,
                                            int r, int y_dtype) {
-  const int lg = lane >> 3, lj = lane & 7;
+  const int lg = lane / G, lj = lane % G;
   const int rb = row0 + lg * RS;                 // this group's first row
   const int nr = max(0, min(RS, rc - rb));
   const int xq4 = rowb;                          // K / 4: distance between the four block quarters
@@ -168,31 +171,30 @@ __device__ __forceinline__ void gs_task_lg(const uint8_t* wbase, int rc, int row
   const int8_t* xp = xs + 16 * lj;
   if (nr == RS) {
 #pragma unroll 2
-    for (int c = lj; c < nchunk; c += 8) {
+    for (int c = lj; c < nchunk; c += G) {
       uint4 w[RS];
 #pragma unroll
       for (int i = 0; i < RS; ++i) w[i] = *reinterpret_cast<const uint4*>(wrow + i * rowb);
       body(w, xp);
-      wrow += 128;
-      xp += 128;
+      wrow += 16 * G;
+      xp += 16 * G;
     }
   } else if (nr > 0) {
-    for (int c = lj; c < nchunk; c += 8) {
+    for (int c = lj; c < nchunk; c += G) {
       uint4 w[RS];
 #pragma unroll
       for (int i = 0; i < RS; ++i)
         w[i] = (i < nr) ? *reinterpret_cast<const uint4*>(wrow + i * rowb) : make_uint4(0u, 0u, 0u, 0u);
       body(w, xp);
-      wrow += 128;
-      xp += 128;
+      wrow += 16 * G;
+      xp += 16 * G;
     }
   }
 #pragma unroll
   for (int i = 0; i < RS; ++i) {
     int t = a[i][0] + (a[i][1] >> 2) + (a[i][2] >> 4) + (a[i][3] >> 6);
-    t += __shfl_xor_sync(0xffffffffu, t, 4);
-    t += __shfl_xor_sync(0xffffffffu, t, 2);
-    t += __shfl_xor_sync(0xffffffffu, t, 1);
+#pragma unroll
+    for (int o = G / 2; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
     a[i][0] = t;
   }
 #pragma unroll
@@ -511,12 +513,18 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
       const uint8_t* wb8 = myslots + slot * p.slot_bytes;
       const int rows = min(P.rc, cur.r1 - cur.r);
       const int r = cur.r;
-      if (MT == 1 && P.task == kGsTaskLG2) {
+      if (MT == 1 && P.task == kGsTaskG8R2) {
         for (int row0 = 0; row0 < rows; row0 += 8)
-          gs_task_lg<2>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
-      } else if (MT == 1 && P.task == kGsTaskLG1) {
+          gs_task_lg<8, 2>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+      } else if (MT == 1 && P.task == kGsTaskG16R2) {
         for (int row0 = 0; row0 < rows; row0 += 4)
-          gs_task_lg<1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+          gs_task_lg<16, 2>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+      } else if (MT == 1 && P.task == kGsTaskG16R1) {
+        for (int row0 = 0; row0 < rows; row0 += 2)
+          gs_task_lg<16, 1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+      } else if (MT == 1 && P.task == kGsTaskG32R1) {
+        for (int row0 = 0; row0 < rows; ++row0)
+          gs_task_lg<32, 1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
       } else {
         constexpr int R = (MT == 1) ? 4 : ((MT == 2) ? 2 : 1);
         const uint32_t* wbase = reinterpret_cast<const uint32_t*>(wb8);

@@ -293,6 +293,40 @@ def run_ours(args):
                          "the previous), programmatic dependent launch, one CUDA graph per step"}
         del cgraph
 
+    # ---- the feed-forward chain: each layer's down projection consumes the
+    # ReLU^2 gate of its up/gate outputs and updates the residual stream ----
+    ffn = None
+    if not args.no_chain:
+        layers = len(stack) // 7
+        hidden = stack[0][0]
+        h = synthetic.activations(1, hidden, seed=replicas.replica_seed(10_000, rank),
+                                  dtype=torch.bfloat16).to(dev)
+        f_calls, f_bytes = [], 0
+        for l in range(layers):
+            (Ku, Nu, Wu, gu), (Kg, Ng, Wg, gg), (Kd, Nd, Wd, gd) = stack[7 * l + 4: 7 * l + 7]
+            yu = torch.empty((1, Nu), dtype=torch.bfloat16, device=dev)
+            yg = torch.empty((1, Ng), dtype=torch.bfloat16, device=dev)
+            upgate = bn.GroupedCall([(h, Wu, gu, gains[Ku], yu), (h, Wg, gg, gains[Kg], yg)], rms_eps=1e-5)
+            f_calls.append((upgate, yg, yu, Wd, gd, gains[Kd], Nd))
+            f_bytes += (Nu * Ku + Ng * Kg + Nd * Kd) // 4 + Ku * 2 + (Nu + Ng) * 2 * 2 + Kd * 2 + Nd * 2 * 2 + 12
+
+        def ffn_step():
+            for upgate, yg, yu, Wd, gd, gaind, Nd in f_calls:
+                upgate()
+                bn.bitnet_linear_relu2(yg, yu, Wd, gd, N=Nd, rms_gain=gaind, rms_eps=1e-5, resid=h, y=h, ws=ws)
+
+        fgraph = capture(ffn_step)
+        fsteps = max(20, args.steps // 10)
+        fms, fms_max, _ = time_graph(fgraph, fsteps, 3)
+        assert bn.bitnet_get_error(ws) == 0
+        ffn = {"value": round(world * f_bytes / (fms_max * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "ms_per_step": round(fms_max, 4), "us_per_layer": round(fms_max * 1e3 / layers, 3),
+               "steps": fsteps, "launches_per_step": 2 * layers, "bytes_per_step": f_bytes,
+               "what": "per layer: up|gate as one grouped launch on the residual stream, then the down "
+                       "projection with the ReLU^2 gate fused into its quantiser and the residual added in "
+                       "its epilogue (bitnet_linear_relu2, in place); 60 dependent launches, one CUDA graph"}
+        del fgraph
+
     # ---- e2e: host buffers, through the public API, no graph ----------------
     e2e = None
     if not args.no_e2e:
@@ -387,6 +421,8 @@ def run_ours(args):
         out["e2e"] = e2e
     if chain is not None:
         out["decode_chain"] = chain
+    if ffn is not None:
+        out["ffn_chain"] = ffn
     if prefill is not None:
         out["prefill"] = prefill
     if cpu is not None:

@@ -26,7 +26,8 @@ PATH_AUTO, PATH_GEMV, PATH_TC = 0, 1, 2
 EXPORTS = ("bitnet_workspace_bytes", "bitnet_quant_weights_workspace_bytes", "bitnet_workspace_init",
            "bitnet_get_error", "bitnet_status_str", "bitnet_quant_weights", "bitnet_ternarise",
            "bitnet_pack", "bitnet_unpack", "bitnet_quant_act", "bitnet_linear", "bitnet_linear_ex",
-           "bitnet_linear_q", "bitnet_linear_grouped", "bitnet_quant_weights_noalloc",
+           "bitnet_linear_q", "bitnet_linear_grouped", "bitnet_linear_relu2", "bitnet_quant_act_relu2",
+           "bitnet_quant_weights_noalloc",
            "bitnet_set_wait_limit_us", "bitnet_watchdog_selftest")
 
 
@@ -68,6 +69,8 @@ def lib() -> ctypes.CDLL:
         "bitnet_pack": ([P, I64, I64, P, P, P], I32),
         "bitnet_unpack": ([P, I64, I64, P, P, P], I32),
         "bitnet_quant_act": ([P, I32, I64, I64, P, F, P, P, P, P], I32),
+        "bitnet_quant_act_relu2": ([P, P, I32, I64, I64, P, F, P, P, P, P], I32),
+        "bitnet_linear_relu2": ([P, P, I32, I64, I64, P, I64, P, P, F, P, P, I32, P, SZ, P], I32),
         "bitnet_linear": ([P, I32, I64, I64, P, I64, P, P, F, P, I32, P, SZ, P], I32),
         "bitnet_linear_ex": ([P, I32, I64, I64, P, I64, P, P, F, P, I32, P, SZ, I32, P], I32),
         "bitnet_linear_q": ([P, P, P, I64, I64, P, I64, P, P, I32, P, P, SZ, I32, P], I32),
@@ -255,6 +258,44 @@ def bitnet_linear(x: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N: int
     _check(lib().bitnet_linear_ex(_ptr(x), _xdtype(x), M, K, _ptr(Wp), N, _ptr(gamma), _ptr(rms_gain),
                                   float(rms_eps), _ptr(y), _ydtype(y.dtype), _ptr(ws), ws.numel(), int(path),
                                   _stream(stream)), "bitnet_linear")
+    return y
+
+
+def bitnet_quant_act_relu2(gate: torch.Tensor, up: torch.Tensor, rms_gain: torch.Tensor | None = None,
+                           rms_eps: float = 1e-5, xq=None, x_scale=None, x_sum=None, stream=None):
+    """Codes, scales and code sums of t = max(gate, 0)^2 * up."""
+    M, K = gate.shape
+    if up.shape != gate.shape or up.dtype != gate.dtype:
+        raise ValueError("gate and up must have the same shape and dtype")
+    if xq is None:
+        xq = torch.empty((M, K), dtype=torch.int8, device=gate.device)
+    if x_scale is None:
+        x_scale = torch.empty(M, dtype=torch.float32, device=gate.device)
+    if x_sum is None:
+        x_sum = torch.empty(M, dtype=torch.int32, device=gate.device)
+    _check(lib().bitnet_quant_act_relu2(_ptr(gate), _ptr(up), _xdtype(gate), M, K, _ptr(rms_gain), float(rms_eps),
+                                        _ptr(xq), _ptr(x_scale), _ptr(x_sum), _stream(stream)),
+           "bitnet_quant_act_relu2")
+    return xq, x_scale, x_sum
+
+
+def bitnet_linear_relu2(gate: torch.Tensor, up: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor,
+                        N: int | None = None, rms_gain: torch.Tensor | None = None, rms_eps: float = 1e-5,
+                        resid: torch.Tensor | None = None, y=None, y_dtype=torch.bfloat16, ws=None, stream=None):
+    """Down projection of the ReLU^2-gated input, plus an optional residual."""
+    M, K = gate.shape
+    if up.shape != gate.shape or up.dtype != gate.dtype:
+        raise ValueError("gate and up must have the same shape and dtype")
+    N = Wp.shape[0] if N is None else N
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype if resid is None else resid.dtype, device=gate.device)
+    if resid is not None and (resid.shape != (M, N) or resid.dtype != y.dtype):
+        raise ValueError("resid must be [M, N] of y's dtype")
+    if ws is None:
+        ws = new_workspace(bitnet_workspace_bytes(M, K, N), gate.device)
+    _check(lib().bitnet_linear_relu2(_ptr(gate), _ptr(up), _xdtype(gate), M, K, _ptr(Wp), N, _ptr(gamma),
+                                     _ptr(rms_gain), float(rms_eps), _ptr(resid), _ptr(y), _ydtype(y.dtype),
+                                     _ptr(ws), ws.numel(), _stream(stream)), "bitnet_linear_relu2")
     return y
 
 

@@ -158,21 +158,39 @@ __device__ __forceinline__ int xs_blocked(int k, int K) {
   return (g & 3) * (K >> 2) + ((g >> 2) << 4) + (k & 15);
 }
 
-// Quantise rows 0..M-1 (M <= MT, K % 16 == 0) of x with one CTA of NT
+// ReLU^2 gate of the feed-forward layers: the down projection's input is
+// t = max(g, 0)^2 * u for the gate and up projections' outputs g and u, in
+// binary32 with one rounding per operation: (r * r) * u.  v holds g on entry.
+template <bool SMEM_SRC = false>
+__device__ __forceinline__ void relu2_gate8(const char* up_row, int x_dtype, int k, float (&v)[8]) {
+  uint4 raw[2];
+  load8raw<SMEM_SRC>(up_row, x_dtype, k, raw);
+  float u[8];
+  decode8(raw, x_dtype, u);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float r = fmaxf(v[i], 0.0f);
+    v[i] = __fmul_rn(__fmul_rn(r, r), u[i]);
+  }
+}
+
+// Quantise rows 0..M-1 (M <= MT, K % 16 == 0) with one CTA of NT
 // threads.  Pass 1 finds max|t| (and sum x^2 with a gain) per row, keeping
 // up to C 8-element bfloat16 chunks per thread in registers; one
 // __syncthreads combines the per-warp partials in a fixed order.  Pass 2
 // writes the codes to dst (row stride dst_stride, generic address) and
 // leaves per-warp partial code sums in S.qpart: the caller's next
 // __syncthreads publishes both.  scale[m] is returned to every thread.
-// The group is threads [tid_base, tid_base + NT) of the block.
+// The group is threads [tid_base, tid_base + NT) of the block.  With x2
+// (same layout as x), the input is the ReLU^2 gate of x (gate) and x2 (up).
 template <int NT, int MT, int C, bool SMEM_SRC = false, int BAR = 0, bool SWZ = false>
 __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dtype, int64_t row_bytes, int M,
                                            int K, const float* __restrict__ gain, float rms_eps, int8_t* dst,
                                            int64_t dst_stride, QuantScratch<NT, MT>& S, float (&scale)[MT],
-                                           int tid_base = 0, bool blocked = false) {
+                                           int tid_base = 0, bool blocked = false,
+                                           const char* __restrict__ x2 = nullptr) {
   const int tid = static_cast<int>(threadIdx.x) - tid_base, lane = tid & 31, warp = tid >> 5;
-  const bool cache_ok = (x_dtype == BITNET_BF16);
+  const bool cache_ok = (x_dtype == BITNET_BF16) && x2 == nullptr;
   uint4 cache[MT][C];
   float am[MT];
   double ss[MT];
@@ -205,6 +223,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
           if (cache_ok) cache[m][c] = raw[0];
           float v[8];
           decode8(raw, x_dtype, v);
+          if (x2 != nullptr) relu2_gate8<SMEM_SRC>(x2 + m * row_bytes, x_dtype, k, v);
           process(v, k);
         }
       }
@@ -214,6 +233,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
         load8raw<SMEM_SRC>(row, x_dtype, k, raw);
         float v[8];
         decode8(raw, x_dtype, v);
+        if (x2 != nullptr) relu2_gate8<SMEM_SRC>(x2 + m * row_bytes, x_dtype, k, v);
         process(v, k);
       }
     }
@@ -283,6 +303,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
             load8raw<SMEM_SRC>(row, x_dtype, k, raw);
           float v[8];
           decode8(raw, x_dtype, v);
+          if (x2 != nullptr) relu2_gate8<SMEM_SRC>(x2 + m * row_bytes, x_dtype, k, v);
           emit(v, k);
         }
       }
@@ -292,6 +313,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
         load8raw<SMEM_SRC>(row, x_dtype, k, raw);
         float v[8];
         decode8(raw, x_dtype, v);
+        if (x2 != nullptr) relu2_gate8<SMEM_SRC>(x2 + m * row_bytes, x_dtype, k, v);
         emit(v, k);
       }
     }
@@ -303,10 +325,12 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
 constexpr int kActThreads = 256;
 
 // One CTA per row.
+// With x2: quantise the ReLU^2 gate of x (gate) and x2 (up).
 __global__ void __launch_bounds__(kActThreads) quant_act_kernel(const void* __restrict__ x, int x_dtype, int K,
                                                                 const float* __restrict__ gain, float rms_eps,
                                                                 int8_t* __restrict__ xq, float* __restrict__ x_scale,
-                                                                int32_t* __restrict__ x_sum) {
+                                                                int32_t* __restrict__ x_sum,
+                                                                const void* __restrict__ x2) {
   __shared__ QuantScratch<kActThreads, 1> S;
   pdl_launch_dependents();
   pdl_wait();
@@ -314,7 +338,8 @@ __global__ void __launch_bounds__(kActThreads) quant_act_kernel(const void* __re
   const int64_t esz = (x_dtype == BITNET_BF16) ? 2 : 4;
   float sc[1];
   quant_rows<kActThreads, 1, 2>(static_cast<const char*>(x) + m * K * esz, x_dtype, K * esz, 1, K, gain, rms_eps,
-                                xq + m * K, K, S, sc);
+                                xq + m * K, K, S, sc, 0, false,
+                                x2 != nullptr ? static_cast<const char*>(x2) + m * K * esz : nullptr);
   __syncthreads();
   if (threadIdx.x == 0) {
     int t = 0;

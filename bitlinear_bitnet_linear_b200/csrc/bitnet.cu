@@ -250,6 +250,8 @@ struct StreamProblem {
   void* y;
   int32_t* acc;
   int64_t K, N;
+  const void* x2;      // up projection of a ReLU^2-gated input (x is the gate), or nullptr
+  const void* resid;   // residual added to y, or nullptr
 };
 
 template <int MAXP>
@@ -329,6 +331,8 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
     g.x_scale = pr[i].x_scale;
     g.y = pr[i].y;
     g.acc = pr[i].acc;
+    g.x2 = pr[i].x2;
+    g.resid = pr[i].resid;
     g.K = static_cast<int>(pr[i].K);
     g.N = static_cast<int>(pr[i].N);
     const int64_t rowb = pr[i].K / 4;
@@ -604,16 +608,36 @@ bitnet_status bitnet_quant_act(const void* x, int x_dtype, int64_t M, int64_t K,
   if (s != BITNET_OK) return s;
   cudaError_t e = launch_pdl(quant_act_kernel, dim3(static_cast<unsigned>(M)), dim3(kActThreads), 0,
                              reinterpret_cast<cudaStream_t>(stream), x, x_dtype, static_cast<int>(K), rms_gain,
-                             rms_eps, xq, x_scale, x_sum);
+                             rms_eps, xq, x_scale, x_sum, static_cast<const void*>(nullptr));
+  return launch_result(e);
+}
+
+bitnet_status bitnet_quant_act_relu2(const void* gate, const void* up, int x_dtype, int64_t M, int64_t K,
+                                     const float* rms_gain, float rms_eps, int8_t* xq, float* x_scale,
+                                     int32_t* x_sum, bitnet_stream_t stream) {
+  if (gate == nullptr || up == nullptr || xq == nullptr || x_scale == nullptr) return BITNET_ERR_NULL;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (check_shape(M, K, 1) != BITNET_OK) return BITNET_ERR_SHAPE;
+  if (!aligned16(gate) || !aligned16(up) || !aligned16(xq) || (rms_gain != nullptr && !aligned16(rms_gain)))
+    return BITNET_ERR_ALIGN;
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  cudaError_t e = launch_pdl(quant_act_kernel, dim3(static_cast<unsigned>(M)), dim3(kActThreads), 0,
+                             reinterpret_cast<cudaStream_t>(stream), gate, x_dtype, static_cast<int>(K), rms_gain,
+                             rms_eps, xq, x_scale, x_sum, up);
   return launch_result(e);
 }
 
 static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in, const float* scale_in,
                                  const int32_t* sum_in, int64_t M, int64_t K, const uint8_t* Wp, int64_t N,
                                  const float* gamma, const float* rms_gain, float rms_eps, void* y, int y_dtype,
-                                 int32_t* acc, void* ws, size_t ws_bytes, int path, cudaStream_t st) {
+                                 int32_t* acc, void* ws, size_t ws_bytes, int path, cudaStream_t st,
+                                 const void* x2 = nullptr, const void* resid = nullptr) {
   if (Wp == nullptr || gamma == nullptr || ws == nullptr) return BITNET_ERR_NULL;
   if (y == nullptr && acc == nullptr) return BITNET_ERR_NULL;
+  if (resid != nullptr && y == nullptr) return BITNET_ERR_NULL;
+  if ((x2 != nullptr && !aligned16(x2)) || (resid != nullptr && !aligned16(resid))) return BITNET_ERR_ALIGN;
   if (y != nullptr && y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
   bitnet_status s = check_shape(M, K, N);
   if (s != BITNET_OK) return s;
@@ -630,11 +654,15 @@ static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in
 
   GemvPlan gp;
   bool gemv_ok = plan_gemv(d, M, K, N, gp) == BITNET_OK;
+  // the gated input and the residual are in the streaming GEMV (K % 64 == 0)
+  // and the tensor-core path, not in the padded-row GEMV
+  if ((x2 != nullptr || resid != nullptr) && K % 64 != 0) gemv_ok = false;
   if (path == BITNET_PATH_GEMV && !gemv_ok) return BITNET_ERR_UNSUPPORTED;
   const bool use_gemv = (path == BITNET_PATH_GEMV) || (path == BITNET_PATH_AUTO && gemv_ok);
 
   if (use_gemv && K % 64 == 0) {
-    StreamProblem sp{x != nullptr ? x : static_cast<const void*>(xq_in), Wp, gamma, rms_gain, scale_in, y, acc, K, N};
+    StreamProblem sp{x != nullptr ? x : static_cast<const void*>(xq_in), Wp, gamma, rms_gain, scale_in, y, acc, K, N,
+                     x2, resid};
     auto* pl = new (std::nothrow) StreamPlan<kStreamSmallP>;
     if (pl == nullptr) return BITNET_ERR_CUDA;
     s = plan_stream<kStreamSmallP>(d, &sp, 1, M, x != nullptr ? x_dtype : BITNET_F32, x == nullptr, rms_eps,
@@ -677,7 +705,7 @@ static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in
     if (ws_bytes < linear_ws_bytes(M, K)) return BITNET_ERR_WORKSPACE;
     LinearWs w = carve(ws, M, K);
     cudaError_t e = launch_pdl(quant_act_kernel, dim3(static_cast<unsigned>(M)), dim3(kActThreads), 0, st, x,
-                               x_dtype, static_cast<int>(K), rms_gain, rms_eps, w.xq, w.scale, w.sum);
+                               x_dtype, static_cast<int>(K), rms_gain, rms_eps, w.xq, w.scale, w.sum, x2);
     if (e != cudaSuccess) return launch_result(e);
     xq = w.xq;
     scale = w.scale;
@@ -692,6 +720,7 @@ static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in
   }
   TcParams p;
   p.Wp = Wp;
+  p.resid = resid;
   p.gamma = gamma;
   p.x_scale = scale;
   p.x_sum = sum;
@@ -723,6 +752,17 @@ bitnet_status bitnet_linear(const void* x, int x_dtype, int64_t M, int64_t K, co
                             size_t ws_bytes, bitnet_stream_t stream) {
   return bitnet_linear_ex(x, x_dtype, M, K, Wp, N, gamma, rms_gain, rms_eps, y, y_dtype, ws, ws_bytes,
                           BITNET_PATH_AUTO, stream);
+}
+
+bitnet_status bitnet_linear_relu2(const void* gate, const void* up, int x_dtype, int64_t M, int64_t K,
+                                  const uint8_t* Wp, int64_t N, const float* gamma, const float* rms_gain,
+                                  float rms_eps, const void* resid, void* y, int y_dtype, void* ws, size_t ws_bytes,
+                                  bitnet_stream_t stream) {
+  if (gate == nullptr || up == nullptr || y == nullptr) return BITNET_ERR_NULL;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (!aligned16(gate)) return BITNET_ERR_ALIGN;
+  return linear_impl(gate, x_dtype, nullptr, nullptr, nullptr, M, K, Wp, N, gamma, rms_gain, rms_eps, y, y_dtype,
+                     nullptr, ws, ws_bytes, BITNET_PATH_AUTO, reinterpret_cast<cudaStream_t>(stream), up, resid);
 }
 
 bitnet_status bitnet_linear_q(const int8_t* xq, const float* x_scale, const int32_t* x_sum, int64_t M, int64_t K,

@@ -295,6 +295,12 @@ __device__ __forceinline__ uint16_t bf16_bits_rne(float f) {
   return static_cast<uint16_t>((u + 0x7FFFu + ((u >> 16) & 1u)) >> 16);
 }
 
+// An element of a y-typed tensor (the residual input) as binary32.
+__device__ __forceinline__ float load_y(const void* y, int y_dtype, int64_t idx) {
+  if (y_dtype == BITNET_BF16) return __uint_as_float(static_cast<uint32_t>(static_cast<const uint16_t*>(y)[idx]) << 16);
+  return static_cast<const float*>(y)[idx];
+}
+
 __device__ __forceinline__ void store_y(void* y, int y_dtype, int64_t idx, float v) {
   if (y_dtype == BITNET_BF16)
     reinterpret_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v);

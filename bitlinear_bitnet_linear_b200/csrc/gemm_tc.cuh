@@ -38,6 +38,7 @@ constexpr int kTcBN = 128;        // weight rows per CTA tile (MMA M)
 
 struct TcParams {
   const uint8_t* Wp;
+  const void* resid;     // [M, N] residual added to y (y_dtype), or nullptr
   const float* gamma;
   const float* x_scale;
   const int32_t* x_sum;
@@ -273,7 +274,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const int a = static_cast<int>(v[i]) - xsi;
             const int64_t idx = static_cast<int64_t>(m) * p.N + n;
             if (p.acc != nullptr) p.acc[idx] = a;
-            if (p.y != nullptr) store_y(p.y, p.y_dtype, idx, __fmul_rn(__int2float_rn(a), gsi));
+            if (p.y != nullptr) {
+              float o = __fmul_rn(__int2float_rn(a), gsi);
+              if (p.resid != nullptr) o = __fadd_rn(load_y(p.resid, p.y_dtype, idx), o);
+              store_y(p.y, p.y_dtype, idx, o);
+            }
           }
         }
       }
@@ -513,7 +518,8 @@ __global__ void __launch_bounds__(kTpThreads, 1)
     const int row = h * 128 + q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     constexpr int kChunks = BM / 32;
-    const bool fast = p.y != nullptr && p.acc == nullptr && p.y_dtype == BITNET_BF16 && p.K <= 32768;
+    const bool fast = p.y != nullptr && p.acc == nullptr && p.resid == nullptr && p.y_dtype == BITNET_BF16 &&
+                      p.K <= 32768;
     pdl_wait();   // token scales and sums come from the previous kernel
     const float gamma = __ldg(p.gamma);
     const float* __restrict__ xsc = p.x_scale;
@@ -582,7 +588,11 @@ __global__ void __launch_bounds__(kTpThreads, 1)
               const int acc = static_cast<int>(v[t]) - xst;
               const int64_t idx = static_cast<int64_t>(m) * p.N + n;
               if (p.acc != nullptr) p.acc[idx] = acc;
-              if (p.y != nullptr) store_y(p.y, p.y_dtype, idx, __fmul_rn(__int2float_rn(acc), gst));
+              if (p.y != nullptr) {
+                float o = __fmul_rn(__int2float_rn(acc), gst);
+                if (p.resid != nullptr) o = __fadd_rn(load_y(p.resid, p.y_dtype, idx), o);
+                store_y(p.y, p.y_dtype, idx, o);
+              }
             }
           }
         }

@@ -54,6 +54,8 @@ constexpr int kGsTaskWarp = 4;      // whole warp over R = 4 / 2 / 1 rows (M = 1
 
 struct GsProblem {
   const void* x;          // [M, K] raw activations (x_dtype) or int8 codes (prequant)
+  const void* x2;         // [M, K] up projection for a ReLU^2-gated input (x is the gate), or nullptr
+  const void* resid;      // [M, N] residual added to y (y_dtype), or nullptr
   const uint8_t* Wp;      // [N, K/4]
   const float* gamma;     // device scalar
   const float* gain;      // [K] RMSNorm gain or nullptr
@@ -203,7 +205,11 @@ __device__ __forceinline__ void gs_task_lg(const uint8_t* wbase, int rc, int row
       const int64_t n = r + rb + i;
       const int accv = a[i][0] - xsum0;
       if (P.acc != nullptr) P.acc[n] = accv;
-      if (P.y != nullptr) store_y(P.y, y_dtype, n, __fmul_rn(__int2float_rn(accv), gs0));
+      if (P.y != nullptr) {
+        float o = __fmul_rn(__int2float_rn(accv), gs0);
+        if (P.resid != nullptr) o = __fadd_rn(load_y(P.resid, y_dtype, n), o);
+        store_y(P.y, y_dtype, n, o);
+      }
     }
   }
 }
@@ -267,7 +273,11 @@ __device__ __forceinline__ void gs_task_warp(const uint32_t* wbase, int rc, int 
         const int accv = a[i][m][0] - xsum[m];
         const int64_t idx = static_cast<int64_t>(m) * P.N + n;
         if (P.acc != nullptr) P.acc[idx] = accv;
-        if (P.y != nullptr) store_y(P.y, y_dtype, idx, __fmul_rn(__int2float_rn(accv), __fmul_rn(gamma, sc[m])));
+        if (P.y != nullptr) {
+          float o = __fmul_rn(__int2float_rn(accv), __fmul_rn(gamma, sc[m]));
+          if (P.resid != nullptr) o = __fadd_rn(load_y(P.resid, y_dtype, idx), o);
+          store_y(P.y, y_dtype, idx, o);
+        }
       }
     }
 }
@@ -297,8 +307,9 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
     r1 = (q == pe) ? re : p.prob[q].N;
   };
   auto shares_x = [&](int q) {   // segment q reuses segment q-1's quantised activations
-    return q > pb && p.prob[q].x == p.prob[q - 1].x && p.prob[q].gain == p.prob[q - 1].gain &&
-           p.prob[q].K == p.prob[q - 1].K && p.prob[q].x_scale == p.prob[q - 1].x_scale;
+    return q > pb && p.prob[q].x == p.prob[q - 1].x && p.prob[q].x2 == p.prob[q - 1].x2 &&
+           p.prob[q].gain == p.prob[q - 1].gain && p.prob[q].K == p.prob[q - 1].K &&
+           p.prob[q].x_scale == p.prob[q - 1].x_scale;
   };
   // Move a cursor `steps` chunks forward through the CTA's segments.
   auto advance = [&](GsCursor& c, int steps) {
@@ -407,7 +418,8 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
       ok = copy_codes(P, xs, Kp, sc, &H.q.qpart[0][0], kAll, 0, tid == CW * 32) && ok;
     } else {
       quant_rows<kAll, MT, 1, false, kGsBarAll, false>(static_cast<const char*>(P.x), p.x_dtype, P.K * esz, p.M,
-                                                      P.K, P.gain, p.rms_eps, xs, Kp, H.q, sc, 0, p.blocked != 0);
+                                                      P.K, P.gain, p.rms_eps, xs, Kp, H.q, sc, 0, p.blocked != 0,
+                                                      static_cast<const char*>(P.x2));
     }
     group_sync<kGsBarAll, kAll>();
     // the activation warp publishes the version; it reads the shared partials
@@ -454,7 +466,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
       } else {
         quant_rows<32, MT, 1, false, kGsBarX, false>(static_cast<const char*>(P.x), p.x_dtype, P.K * esz, p.M,
                                                      P.K, P.gain, p.rms_eps, xs, Kp, H.qx, sc, CW * 32,
-                                                     p.blocked != 0);
+                                                     p.blocked != 0, static_cast<const char*>(P.x2));
       }
       __syncwarp();
       if (lane == 0) {

@@ -201,6 +201,33 @@ bitnet_status bitnet_linear_q(const int8_t *xq, const float *x_scale, const int3
                               const float *gamma, void *y, int y_dtype, int32_t *acc,
                               void *ws, size_t ws_bytes, int path, bitnet_stream_t stream);
 
+/* Feed-forward down projection with the ReLU^2 gate fused into the input
+ * quantiser ("Key Technologies ...", Architectural Innovations: squared
+ * ReLU activations in the feed-forward layers, no bias):
+ *   t_k = (max(gate_k, 0) * max(gate_k, 0)) * up_k   (binary32, one rounding
+ *         per operation, in that order; NaN gate counts as 0)
+ * then t is quantised and contracted exactly as x in bitnet_linear (with
+ * the optional RMSNorm gain applied to t), and
+ *   y[m,n] = resid[m,n] + (float)acc[m,n] * (gamma * s_x[m])   (binary32
+ *            sum of the rounded product, then y_dtype)
+ * when resid (the block's residual stream, [M, N] of y_dtype) is given,
+ * else y as in bitnet_linear.  gate, up: [M, K] of x_dtype (the gate and up
+ * projections' outputs).  resid may alias y.  Same workspace as
+ * bitnet_linear.  The residual add is this library's reading of a
+ * Transformer feed-forward block; the pages name only the gate. */
+bitnet_status bitnet_linear_relu2(const void *gate, const void *up, int x_dtype, int64_t M, int64_t K,
+                                  const uint8_t *Wp, int64_t N, const float *gamma,
+                                  const float *rms_gain, float rms_eps, const void *resid,
+                                  void *y, int y_dtype, void *ws, size_t ws_bytes,
+                                  bitnet_stream_t stream);
+
+/* bitnet_quant_act of the ReLU^2 gate t = max(gate, 0)^2 * up (as in
+ * bitnet_linear_relu2): codes, scales and code sums of t. */
+bitnet_status bitnet_quant_act_relu2(const void *gate, const void *up, int x_dtype, int64_t M, int64_t K,
+                                     const float *rms_gain, float rms_eps,
+                                     int8_t *xq, float *x_scale, int32_t *x_sum,
+                                     bitnet_stream_t stream);
+
 /* One problem of a grouped GEMV call. */
 typedef struct bitnet_gemv_problem {
     const void *x;          /* [M, K] activations of the call's x_dtype, device */

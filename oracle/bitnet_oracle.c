@@ -19,6 +19,8 @@
  *              the ternary dot product as "sum of activations where the
  *              weight is +1 minus sum where it is -1", and "activations are
  *              int8 during inference".
+ *   [KeyTech] also gives the feed-forward activation (squared ReLU, the
+ *              ReLU^2 gate below).
  *   [Notes]    "BitNet Technical Notes" (afondiel.github.io), "System
  *              Design" / Appendix glossary: bit-packing at 2 bits per
  *              ternary weight.
@@ -281,6 +283,41 @@ void orc_output(const int32_t *acc, int64_t M, int64_t N, float gamma,
         float sm = gamma * scale[m];
         for (int64_t n = 0; n < N; ++n)
             y[m * N + n] = (float)acc[m * N + n] * sm;
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* ReLU^2 gate of the feed-forward layers.  [KeyTech] "Architectural        */
+/* Innovations": squared ReLU activations in the feed-forward layers.  The  */
+/* down projection's input is the gate projection's output squared after    */
+/* ReLU, times the up projection's output:                                  */
+/*   t = (r * r) * u,  r = max(g, 0)                                        */
+/* in binary32, one rounding per operation, in that order.  A NaN gate      */
+/* counts as 0 (the comparison g > 0 is false).                             */
+/* ------------------------------------------------------------------------ */
+void orc_relu2_gate(const float *gate, const float *up, int64_t n, float *t)
+{
+    for (int64_t i = 0; i < n; ++i) {
+        float g = gate[i];
+        float r = (g > 0.0f) ? g : 0.0f;
+        float rr = r * r;
+        t[i] = rr * up[i];
+    }
+}
+
+/* Output with the block's residual stream added (a Transformer feed-forward */
+/* block adds its output to its input; the pages name only the gate):       */
+/*   y[m,n] = resid[m,n] + (float)acc[m,n] * (gamma * s[m])                 */
+/* binary32: the product rounded, then the sum rounded.                      */
+void orc_output_resid(const int32_t *acc, int64_t M, int64_t N, float gamma,
+                      const float *scale, const float *resid, float *y)
+{
+    for (int64_t m = 0; m < M; ++m) {
+        float sm = gamma * scale[m];
+        for (int64_t n = 0; n < N; ++n) {
+            float prod = (float)acc[m * N + n] * sm;
+            y[m * N + n] = resid[m * N + n] + prod;
+        }
     }
 }
 

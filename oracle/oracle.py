@@ -58,6 +58,8 @@ def lib():
         L.orc_linear_i32.argtypes = [P, I64, I64, P, I64, P]; L.orc_linear_i32.restype = None
         L.orc_output.argtypes = [P, I64, I64, F, P, P]; L.orc_output.restype = None
         L.orc_to_bf16.argtypes = [P, I64, P]; L.orc_to_bf16.restype = None
+        L.orc_relu2_gate.argtypes = [P, P, I64, P]; L.orc_relu2_gate.restype = None
+        L.orc_output_resid.argtypes = [P, I64, I64, F, P, P, P]; L.orc_output_resid.restype = None
         _lib = L
     return _lib
 
@@ -150,6 +152,28 @@ def output(acc: np.ndarray, g: float, scale: np.ndarray) -> np.ndarray:
     M, N = acc.shape
     y = np.empty((M, N), np.float32)
     lib().orc_output(_p(acc), M, N, float(np.float32(g)), _p(scale), _p(y))
+    return y
+
+
+def relu2_gate(gate: np.ndarray, up: np.ndarray) -> np.ndarray:
+    """t = max(gate, 0)^2 * up in binary32, (r * r) * u."""
+    gate = _c(gate, np.float32)
+    up = _c(up, np.float32)
+    assert gate.shape == up.shape
+    t = np.empty(gate.shape, np.float32)
+    lib().orc_relu2_gate(_p(gate), _p(up), gate.size, _p(t))
+    return t
+
+
+def output_resid(acc: np.ndarray, g: float, scale: np.ndarray, resid: np.ndarray) -> np.ndarray:
+    """y = resid + acc * (gamma * s_m) in binary32."""
+    acc = _c(acc, np.int32)
+    scale = _c(scale, np.float32)
+    resid = _c(resid, np.float32)
+    M, N = acc.shape
+    assert resid.shape == (M, N)
+    y = np.empty((M, N), np.float32)
+    lib().orc_output_resid(_p(acc), M, N, float(np.float32(g)), _p(scale), _p(resid), _p(y))
     return y
 
 

@@ -334,3 +334,69 @@ def test_bf16_rounding_matches_torch(orc):
     ours = orc.to_bf16_bits(v)
     ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     assert (ours == ref).all()
+
+
+# ---------------------------------------------------------------------------
+# ReLU^2 gate and residual output ("Key Technologies ...", Architectural
+# Innovations: squared ReLU in the feed-forward layers).
+# ---------------------------------------------------------------------------
+def test_relu2_golden(orc):
+    rows = [ln.split() for ln in golden_lines("relu2_examples.txt")]
+    g = np.array([float(r[0]) for r in rows], np.float32)
+    u = np.array([float(r[1]) for r in rows], np.float32)
+    want = np.array([float(r[2]) for r in rows], np.float32)
+    got = orc.relu2_gate(g, u)
+    assert np.array_equal(got, want), (got, want)
+
+
+def test_relu2_invariants(orc):
+    rng = np.random.default_rng(7)
+    g = rng.standard_normal(20000).astype(np.float32) * 3
+    u = rng.standard_normal(20000).astype(np.float32) * 3
+    t = orc.relu2_gate(g, u)
+    assert np.all(t[g <= 0] == 0)                      # gate closed: no input
+    pos = g > 0
+    assert np.all(np.sign(t[pos]) == np.sign(u[pos]) * (t[pos] != 0))   # sign of the up branch
+    # integer-valued operands small enough to be exact: t is g^2 u exactly
+    gi = rng.integers(-20, 21, 5000).astype(np.float32)
+    ui = rng.integers(-50, 51, 5000).astype(np.float32)
+    ti = orc.relu2_gate(gi, ui)
+    want = np.where(gi > 0, gi.astype(np.int64) ** 2 * ui.astype(np.int64), 0)
+    assert np.array_equal(ti.astype(np.int64), want)
+    # a unit gate passes u through; a power-of-two gate scales u exactly
+    assert np.array_equal(orc.relu2_gate(np.ones(100, np.float32), u[:100]), u[:100])
+    assert np.array_equal(orc.relu2_gate(np.full(100, 4.0, np.float32), u[:100]), u[:100] * np.float32(16))
+
+
+def test_relu2_then_quant_equals_quant_of_product(orc):
+    """Composition by definition: quantising the gate output is quantising t."""
+    rng = np.random.default_rng(8)
+    g = rng.standard_normal((3, 256)).astype(np.float32)
+    u = rng.standard_normal((3, 256)).astype(np.float32)
+    t = orc.relu2_gate(g, u)
+    xq, sc, xs = orc.quant_act(t)
+    # at least one code of every row with a nonzero input is +-127
+    for m in range(3):
+        if np.any(t[m] != 0):
+            assert np.max(np.abs(xq[m])) == 127
+    assert np.array_equal(xs, xq.astype(np.int64).sum(axis=1))
+
+
+def test_output_resid(orc):
+    acc = np.array([[3, -2, 0]], np.int32)
+    scale = np.array([2.0], np.float32)
+    resid = np.array([[1.0, 0.5, -7.25]], np.float32)
+    y = orc.output_resid(acc, 0.5, scale, resid)
+    # gamma * s = 1: y = resid + acc exactly
+    assert np.array_equal(y, np.array([[4.0, -1.5, -7.25]], np.float32))
+    rng = np.random.default_rng(9)
+    acc = rng.integers(-100000, 100000, (4, 64)).astype(np.int32)
+    scale = rng.random(4).astype(np.float32) * 0.01
+    zero = np.zeros((4, 64), np.float32)
+    # zero residual: the plain output; zero accumulator: the residual itself
+    assert np.array_equal(orc.output_resid(acc, 0.0173, scale, zero), orc.output(acc, 0.0173, scale))
+    r = rng.standard_normal((4, 64)).astype(np.float32)
+    assert np.array_equal(orc.output_resid(np.zeros_like(acc), 0.0173, scale, r), r)
+    # one rounding per operation: product rounded, then the sum
+    prod = orc.output(acc, 0.0173, scale)
+    assert np.array_equal(orc.output_resid(acc, 0.0173, scale, r), (r + prod).astype(np.float32))

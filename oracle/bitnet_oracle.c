@@ -21,6 +21,8 @@
  *              int8 during inference".
  *   [KeyTech] also gives the feed-forward activation (squared ReLU, the
  *              ReLU^2 gate below).
+ *   [Gartu] also names the binary variant, BitNet b1 ("BitNet b1 (binaire)":
+ *              weights exactly +1 or -1), restated in orc_binarise below.
  *   [Notes]    "BitNet Technical Notes" (afondiel.github.io), "System
  *              Design" / Appendix glossary: bit-packing at 2 bits per
  *              ternary weight.
@@ -284,6 +286,58 @@ void orc_output(const int32_t *acc, int64_t M, int64_t N, float gamma,
         for (int64_t n = 0; n < N; ++n)
             y[m * N + n] = (float)acc[m * N + n] * sm;
     }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Binary weights (BitNet b1).  [Gartu] "BitNet b1 (binaire)": every weight */
+/* of the BitLinear layer is exactly +1 or -1.  The pages give no rule, so  */
+/* the reading is the sign, ties (zero) to +1: W_b = +1 where W >= 0, else  */
+/* -1 (a NaN compares false and gives -1).  The scale is the same absmean   */
+/* beta = mean|W| as the ternary case (orc_gamma): sign(W) * mean|W| is the */
+/* binary approximation of W with the least sum of squared errors.          */
+/* ------------------------------------------------------------------------ */
+void orc_binarise(const float *W, int64_t n, int8_t *Wb)
+{
+    for (int64_t i = 0; i < n; ++i) Wb[i] = (W[i] >= 0.0f) ? (int8_t)1 : (int8_t)-1;
+}
+
+/* 1-bit pack: bit 1 for +1, 0 for -1.  K is split into groups of 32       */
+/* weights, one little-endian uint32 each (group g of row n at byte offset  */
+/* n*K/8 + 4g); weight k = 32g + 4s + j (s in 0..7, j in 0..3) sits at bit  */
+/* 8j + s, so (word >> s) & 0x01010101 holds the bits of k = 32g+4s .. +3    */
+/* one per byte in order.  Values other than +-1 are stored as 0 (-1) and   */
+/* counted.  Requires K % 32 == 0.                                          */
+int64_t orc_pack_b1(const int8_t *Wb, int64_t N, int64_t K, uint8_t *Wp)
+{
+    int64_t bad = 0;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < K / 32; ++g) {
+            uint32_t word = 0;
+            for (int s = 0; s < 8; ++s)
+                for (int j = 0; j < 4; ++j) {
+                    int8_t v = Wb[n * K + 32 * g + 4 * s + j];
+                    if (v != 1 && v != -1) ++bad;
+                    if (v == 1) word |= 1u << (8 * j + s);
+                }
+            uint8_t *o = Wp + n * (K / 8) + 4 * g;
+            o[0] = (uint8_t)(word & 0xff);
+            o[1] = (uint8_t)((word >> 8) & 0xff);
+            o[2] = (uint8_t)((word >> 16) & 0xff);
+            o[3] = (uint8_t)(word >> 24);
+        }
+    return bad;
+}
+
+void orc_unpack_b1(const uint8_t *Wp, int64_t N, int64_t K, int8_t *Wb)
+{
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < K / 32; ++g) {
+            const uint8_t *b = Wp + n * (K / 8) + 4 * g;
+            uint32_t word = (uint32_t)b[0] | ((uint32_t)b[1] << 8) | ((uint32_t)b[2] << 16) | ((uint32_t)b[3] << 24);
+            for (int s = 0; s < 8; ++s)
+                for (int j = 0; j < 4; ++j)
+                    Wb[n * K + 32 * g + 4 * s + j] = ((word >> (8 * j + s)) & 1u) ? (int8_t)1 : (int8_t)-1;
+        }
 }
 
 /* ------------------------------------------------------------------------ */

@@ -59,6 +59,9 @@ def lib():
         L.orc_output.argtypes = [P, I64, I64, F, P, P]; L.orc_output.restype = None
         L.orc_to_bf16.argtypes = [P, I64, P]; L.orc_to_bf16.restype = None
         L.orc_relu2_gate.argtypes = [P, P, I64, P]; L.orc_relu2_gate.restype = None
+        L.orc_binarise.argtypes = [P, I64, P]; L.orc_binarise.restype = None
+        L.orc_pack_b1.argtypes = [P, I64, I64, P]; L.orc_pack_b1.restype = I64
+        L.orc_unpack_b1.argtypes = [P, I64, I64, P]; L.orc_unpack_b1.restype = None
         L.orc_output_resid.argtypes = [P, I64, I64, F, P, P, P]; L.orc_output_resid.restype = None
         _lib = L
     return _lib
@@ -153,6 +156,36 @@ def output(acc: np.ndarray, g: float, scale: np.ndarray) -> np.ndarray:
     y = np.empty((M, N), np.float32)
     lib().orc_output(_p(acc), M, N, float(np.float32(g)), _p(scale), _p(y))
     return y
+
+
+def binarise(W: np.ndarray) -> np.ndarray:
+    """BitNet b1 weights: +1 where W >= 0, else -1 ([Gartu] binary BitLinear)."""
+    W = _c(W, np.float32)
+    out = np.empty(W.shape, np.int8)
+    lib().orc_binarise(_p(W), W.size, _p(out))
+    return out
+
+
+def quant_weights_b1(W: np.ndarray):
+    """(W_b, beta): signs and the absmean scale."""
+    return binarise(W), gamma(W)
+
+
+def pack_b1(Wb: np.ndarray):
+    """1 bit per weight.  Returns (packed [N, K/8] uint8, n_invalid)."""
+    Wb = _c(Wb, np.int8)
+    N, K = Wb.shape
+    out = np.empty((N, K // 8), np.uint8)
+    bad = lib().orc_pack_b1(_p(Wb), N, K, _p(out))
+    return out, int(bad)
+
+
+def unpack_b1(Wp: np.ndarray, K: int) -> np.ndarray:
+    Wp = _c(Wp, np.uint8)
+    N = Wp.shape[0]
+    out = np.empty((N, K), np.int8)
+    lib().orc_unpack_b1(_p(Wp), N, K, _p(out))
+    return out
 
 
 def relu2_gate(gate: np.ndarray, up: np.ndarray) -> np.ndarray:

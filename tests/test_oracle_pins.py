@@ -400,3 +400,66 @@ def test_output_resid(orc):
     # one rounding per operation: product rounded, then the sum
     prod = orc.output(acc, 0.0173, scale)
     assert np.array_equal(orc.output_resid(acc, 0.0173, scale, r), (r + prod).astype(np.float32))
+
+
+# ---------------------------------------------------------------------------
+# BitNet b1 binary weights ("BitNet / Ternary / Binary", BitNet b1 (binaire):
+# every weight exactly +1 or -1).
+# ---------------------------------------------------------------------------
+def test_binarise_sign_rule(orc):
+    W = np.array([[0.3, -0.3, 0.0, -0.0, 1e-30, -1e-30, np.nan, np.inf, -np.inf, 5.0, -2.0, 7.0]], np.float32)
+    want = np.array([[1, -1, 1, 1, 1, -1, -1, 1, -1, 1, -1, 1]], np.int8)
+    assert np.array_equal(orc.binarise(W), want)
+
+
+def test_binarise_scale_and_idempotence(orc):
+    rng = np.random.default_rng(21)
+    B = np.where(rng.random((64, 96)) < 0.5, -1, 1).astype(np.int8)
+    for c in (0.02, 3.0, 2.0 ** -20):
+        W = (B.astype(np.float32) * np.float32(c)).astype(np.float32)
+        Wb, beta = orc.quant_weights_b1(W)
+        assert np.array_equal(Wb, B)                 # signs of a scaled binary matrix come back
+        assert beta == np.float32(c)                 # mean of equal magnitudes is that magnitude
+    # beta is the absmean of the latent weights (the ternary gamma statistic)
+    W = rng.standard_normal((37, 64)).astype(np.float32)
+    assert orc.quant_weights_b1(W)[1] == orc.gamma(W)
+
+
+def test_pack_b1_golden(orc):
+    lines = golden_lines("pack_b1_layout.txt")
+    w = np.array([[int(v) for v in lines[0].split()]], np.int8)
+    want = np.array([[int(v, 16) for v in lines[1].split()]], np.uint8)
+    packed, bad = orc.pack_b1(w)
+    assert bad == 0 and np.array_equal(packed, want)
+
+
+def test_pack_b1_bijection(orc):
+    rng = np.random.default_rng(22)
+    B = np.where(rng.random((16, 256)) < 0.5, -1, 1).astype(np.int8)
+    P, bad = orc.pack_b1(B)
+    assert bad == 0 and P.shape == (16, 32)
+    assert np.array_equal(orc.unpack_b1(P, 256), B)
+    # every byte pattern is a valid packing: unpack then pack is the identity
+    R = rng.integers(0, 256, (8, 64), dtype=np.uint8)
+    assert np.array_equal(orc.pack_b1(orc.unpack_b1(R, 512))[0], R)
+    # each single bit maps to one weight: k = 32g + 4s + j <-> bit 8j + s
+    for bit in range(32):
+        word = np.array([[bit < 8 and 1 << bit or 0, bit >= 8 and bit < 16 and 1 << (bit - 8) or 0,
+                          bit >= 16 and bit < 24 and 1 << (bit - 16) or 0, bit >= 24 and 1 << (bit - 24) or 0]],
+                        np.uint8)
+        w = orc.unpack_b1(word, 32)[0]
+        j, s = bit // 8, bit % 8
+        assert np.flatnonzero(w == 1).tolist() == [4 * s + j]
+    assert orc.pack_b1(np.zeros((1, 32), np.int8))[1] == 32       # non +-1 values counted
+
+
+def test_binary_contraction_add_subtract(orc):
+    """acc = sum over +1 weights minus sum over -1 weights = 2 * sum_{b=1} x - sum x."""
+    rng = np.random.default_rng(23)
+    xq = rng.integers(-127, 128, (5, 128)).astype(np.int8)
+    B = np.where(rng.random((9, 128)) < 0.5, -1, 1).astype(np.int8)
+    acc = orc.linear_i32(xq, B)
+    x = xq.astype(np.int64)
+    plus = (B == 1).astype(np.int64)
+    assert np.array_equal(acc, x @ plus.T - x @ (1 - plus).T)
+    assert np.array_equal(acc, 2 * (x @ plus.T) - x.sum(axis=1, keepdims=True))

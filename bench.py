@@ -327,6 +327,41 @@ def run_ours(args):
                        "its epilogue (bitnet_linear_relu2, in place); 60 dependent launches, one CUDA graph"}
         del fgraph
 
+    # ---- BitNet b1: the same stack with binary weights, 1 bit per weight ----
+    b1 = None
+    if not args.no_chain:
+        b1_stack = []
+        with torch.cuda.stream(stream):
+            for mt in mats:
+                gens.manual_seed(mt.seed)
+                W = torch.randn((mt.N, mt.K), generator=gens, device=dev, dtype=torch.float32) * synthetic.W_SIGMA
+                Wb, beta = bn.bitnet_quant_weights_b1(W)
+                b1_stack.append((bn.bitnet_pack_b1(Wb), beta))
+                del W, Wb
+        torch.cuda.synchronize()
+        b1_call = bn.GroupedCall([(x, Wp1, beta, gains[K], y) for (K, N, _, _), (Wp1, beta), x, y
+                                  in zip(stack, b1_stack, xs, ys)], rms_eps=1e-5, ws=ws, bits=1)
+
+        def b1_steps(n):
+            def fn():
+                for _ in range(n):
+                    b1_call()
+            return fn
+
+        b1_bytes = sum(N * K // 8 + K * 2 + N * 2 + 4 for (K, N, _, _) in stack)
+        b1_graph = capture(b1_steps(per_graph))
+        bsteps = (max(20, args.steps // 2) // per_graph) * per_graph
+        bms, bms_max, _ = time_graph(b1_graph, bsteps // per_graph, 3)
+        bms, bms_max = bms / per_graph, bms_max / per_graph
+        assert bn.bitnet_get_error(ws) == 0
+        b1 = {"value": round(world * b1_bytes / (bms_max * 1e-3) / 1e9, 2), "unit": "GB/s",
+              "ms_per_step": round(bms_max, 5), "tokens_per_s": round(world * 1e3 / bms_max, 1),
+              "bytes_per_step": b1_bytes, "steps": bsteps,
+              "what": "the 210-call stack with BitNet b1 weights (sign, absmean scale, 1 bit per weight, "
+                      "297 MB), one grouped launch per token (bitnet_linear_grouped_b1), CUDA graphs of "
+                      f"{per_graph} steps"}
+        del b1_graph, b1_call, b1_stack
+
     # ---- e2e: host buffers, through the public API, no graph ----------------
     e2e = None
     if not args.no_e2e:
@@ -423,6 +458,8 @@ def run_ours(args):
         out["decode_chain"] = chain
     if ffn is not None:
         out["ffn_chain"] = ffn
+    if b1 is not None:
+        out["b1_decode"] = b1
     if prefill is not None:
         out["prefill"] = prefill
     if cpu is not None:

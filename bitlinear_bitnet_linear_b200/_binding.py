@@ -27,6 +27,8 @@ EXPORTS = ("bitnet_workspace_bytes", "bitnet_quant_weights_workspace_bytes", "bi
            "bitnet_get_error", "bitnet_status_str", "bitnet_quant_weights", "bitnet_ternarise",
            "bitnet_pack", "bitnet_unpack", "bitnet_quant_act", "bitnet_linear", "bitnet_linear_ex",
            "bitnet_linear_q", "bitnet_linear_grouped", "bitnet_linear_relu2", "bitnet_quant_act_relu2",
+           "bitnet_quant_weights_b1", "bitnet_pack_b1", "bitnet_unpack_b1", "bitnet_linear_b1",
+           "bitnet_linear_grouped_b1",
            "bitnet_quant_weights_noalloc",
            "bitnet_set_wait_limit_us", "bitnet_watchdog_selftest")
 
@@ -70,6 +72,11 @@ def lib() -> ctypes.CDLL:
         "bitnet_unpack": ([P, I64, I64, P, P, P], I32),
         "bitnet_quant_act": ([P, I32, I64, I64, P, F, P, P, P, P], I32),
         "bitnet_quant_act_relu2": ([P, P, I32, I64, I64, P, F, P, P, P, P], I32),
+        "bitnet_quant_weights_b1": ([P, I64, I64, P, P, P, SZ, P], I32),
+        "bitnet_pack_b1": ([P, I64, I64, P, P, P], I32),
+        "bitnet_unpack_b1": ([P, I64, I64, P, P], I32),
+        "bitnet_linear_b1": ([P, I32, I64, I64, P, I64, P, P, F, P, I32, P, SZ, P], I32),
+        "bitnet_linear_grouped_b1": ([P, I32, I32, F, I32, P, SZ, P], I32),
         "bitnet_linear_relu2": ([P, P, I32, I64, I64, P, I64, P, P, F, P, P, I32, P, SZ, P], I32),
         "bitnet_linear": ([P, I32, I64, I64, P, I64, P, P, F, P, I32, P, SZ, P], I32),
         "bitnet_linear_ex": ([P, I32, I64, I64, P, I64, P, P, F, P, I32, P, SZ, I32, P], I32),
@@ -261,6 +268,50 @@ def bitnet_linear(x: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N: int
     return y
 
 
+def bitnet_quant_weights_b1(W: torch.Tensor, Wb: torch.Tensor | None = None, beta: torch.Tensor | None = None,
+                            ws: torch.Tensor | None = None, want_wb: bool = True, stream=None):
+    """BitNet b1: (W_b int8 +-1 [N, K] or None, beta float32 [1])."""
+    N, K = W.shape
+    if want_wb and Wb is None:
+        Wb = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    if beta is None:
+        beta = torch.empty(1, dtype=torch.float32, device=W.device)
+    if ws is None:
+        ws = new_workspace(bitnet_quant_weights_workspace_bytes(N, K), W.device)
+    _check(lib().bitnet_quant_weights_b1(_ptr(W), N, K, _ptr(Wb) if want_wb else None, _ptr(beta), _ptr(ws),
+                                         ws.numel(), _stream(stream)), "bitnet_quant_weights_b1")
+    return (Wb if want_wb else None), beta
+
+
+def bitnet_pack_b1(Wb: torch.Tensor, n_invalid: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    N, K = Wb.shape
+    Wp = torch.empty((N, K // 8), dtype=torch.uint8, device=Wb.device)
+    _check(lib().bitnet_pack_b1(_ptr(Wb), N, K, _ptr(Wp), _ptr(n_invalid), _stream(stream)), "bitnet_pack_b1")
+    return Wp
+
+
+def bitnet_unpack_b1(Wp: torch.Tensor, K: int, stream=None) -> torch.Tensor:
+    N = Wp.shape[0]
+    Wb = torch.empty((N, K), dtype=torch.int8, device=Wp.device)
+    _check(lib().bitnet_unpack_b1(_ptr(Wp), N, K, _ptr(Wb), _stream(stream)), "bitnet_unpack_b1")
+    return Wb
+
+
+def bitnet_linear_b1(x: torch.Tensor, Wp: torch.Tensor, beta: torch.Tensor, N: int | None = None,
+                     rms_gain: torch.Tensor | None = None, rms_eps: float = 1e-5, y=None,
+                     y_dtype=torch.bfloat16, ws=None, stream=None):
+    M, K = x.shape
+    N = Wp.shape[0] if N is None else N
+    if y is None:
+        y = torch.empty((M, N), dtype=y_dtype, device=x.device)
+    if ws is None:
+        ws = new_workspace(bitnet_workspace_bytes(M, K, N), x.device)
+    _check(lib().bitnet_linear_b1(_ptr(x), _xdtype(x), M, K, _ptr(Wp), N, _ptr(beta), _ptr(rms_gain),
+                                  float(rms_eps), _ptr(y), _ydtype(y.dtype), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "bitnet_linear_b1")
+    return y
+
+
 def bitnet_quant_act_relu2(gate: torch.Tensor, up: torch.Tensor, rms_gain: torch.Tensor | None = None,
                            rms_eps: float = 1e-5, xq=None, x_scale=None, x_sum=None, stream=None):
     """Codes, scales and code sums of t = max(gate, 0)^2 * up."""
@@ -340,7 +391,7 @@ class GroupedCall:
     """A prepared grouped call: the problem table is built once and reused
     (for CUDA-graph capture or repeated launches)."""
 
-    def __init__(self, problems, rms_eps: float = 1e-5, ws=None):
+    def __init__(self, problems, rms_eps: float = 1e-5, ws=None, bits: int = 2):
         self.arr = (GemvProblem * len(problems))()
         self.M = problems[0][0].shape[0]
         self.xd = _xdtype(problems[0][0])
@@ -351,10 +402,16 @@ class GroupedCall:
                                       None if gain is None else _ptr(gain).value, _ptr(y).value,
                                       x.shape[1], Wp.shape[0])
         self.n = len(problems)
+        self.bits = int(bits)   # 2: ternary codes (bitnet_pack); 1: BitNet b1 signs (bitnet_pack_b1)
         self.eps = float(rms_eps)
         self.ws = ws if ws is not None else new_workspace(256, problems[0][0].device)
 
     def __call__(self, stream=None):
+        if self.bits == 1:
+            _check(lib().bitnet_linear_grouped_b1(ctypes.cast(self.arr, ctypes.c_void_p), self.n, self.xd, self.eps,
+                                                  self.yd, _ptr(self.ws), self.ws.numel(), _stream(stream)),
+                   "bitnet_linear_grouped_b1")
+            return
         _check(lib().bitnet_linear_grouped(ctypes.cast(self.arr, ctypes.c_void_p), self.n, self.M, self.xd,
                                            self.eps, self.yd, _ptr(self.ws), self.ws.numel(), _stream(stream)),
                "bitnet_linear_grouped")

@@ -158,6 +158,14 @@ __device__ __forceinline__ int xs_blocked(int k, int K) {
   return (g & 3) * (K >> 2) + ((g >> 2) << 4) + (k & 15);
 }
 
+// The same with eight quarters, for the 1-bit GEMV (K % 128 == 0): 16-byte
+// block g = 8c + e at e * K/8 + 16 c, the eight blocks that meet one 16-byte
+// load of packed signs (128 weights, chunk c).
+__device__ __forceinline__ int xs_blocked8(int k, int K) {
+  const int g = k >> 4;
+  return (g & 7) * (K >> 3) + ((g >> 3) << 4) + (k & 15);
+}
+
 // ReLU^2 gate of the feed-forward layers: the down projection's input is
 // t = max(g, 0)^2 * u for the gate and up projections' outputs g and u, in
 // binary32 with one rounding per operation: (r * r) * u.  v holds g on entry.
@@ -187,7 +195,7 @@ template <int NT, int MT, int C, bool SMEM_SRC = false, int BAR = 0, bool SWZ = 
 __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dtype, int64_t row_bytes, int M,
                                            int K, const float* __restrict__ gain, float rms_eps, int8_t* dst,
                                            int64_t dst_stride, QuantScratch<NT, MT>& S, float (&scale)[MT],
-                                           int tid_base = 0, bool blocked = false,
+                                           int tid_base = 0, int blocked = 0,
                                            const char* __restrict__ x2 = nullptr) {
   const int tid = static_cast<int>(threadIdx.x) - tid_base, lane = tid & 31, warp = tid >> 5;
   const bool cache_ok = (x_dtype == BITNET_BF16) && x2 == nullptr;
@@ -289,7 +297,7 @@ __device__ __forceinline__ void quant_rows(const char* __restrict__ x, int x_dty
           lo |= (static_cast<uint32_t>(q0) & 0xffu) << (8 * i);
           hi |= (static_cast<uint32_t>(q1) & 0xffu) << (8 * i);
         }
-        const int off = SWZ ? xs_swizzle(k) : (blocked ? xs_blocked(k, K) : k);
+        const int off = SWZ ? xs_swizzle(k) : (blocked == 1 ? xs_blocked(k, K) : (blocked == 2 ? xs_blocked8(k, K) : k));
         *reinterpret_cast<uint2*>(drow + off) = make_uint2(lo, hi);
       };
 #pragma unroll
@@ -338,7 +346,7 @@ __global__ void __launch_bounds__(kActThreads) quant_act_kernel(const void* __re
   const int64_t esz = (x_dtype == BITNET_BF16) ? 2 : 4;
   float sc[1];
   quant_rows<kActThreads, 1, 2>(static_cast<const char*>(x) + m * K * esz, x_dtype, K * esz, 1, K, gain, rms_eps,
-                                xq + m * K, K, S, sc, 0, false,
+                                xq + m * K, K, S, sc, 0, 0,
                                 x2 != nullptr ? static_cast<const char*>(x2) + m * K * esz : nullptr);
   __syncthreads();
   if (threadIdx.x == 0) {

@@ -262,7 +262,7 @@ struct StreamPlan {
 
 template <int MAXP>
 bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int count, int64_t M, int x_dtype,
-                          bool prequant, float rms_eps, int y_dtype, StreamPlan<MAXP>& pl) {
+                          bool prequant, float rms_eps, int y_dtype, StreamPlan<MAXP>& pl, int bits = 2) {
   if (count < 1 || count > MAXP || M < 1 || M > kGemvMaxM) return BITNET_ERR_UNSUPPORTED;
   GsParams<MAXP>& p = pl.p;
   pl.MT = M <= 1 ? 1 : (M <= 2 ? 2 : 4);
@@ -274,10 +274,11 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
   p.rms_eps = rms_eps;
   int64_t total = 0, max_rowb = 0, Kmax = 0, xmax = 0;
   const int64_t esz = prequant ? 1 : (x_dtype == BITNET_BF16 ? 2 : 4);
+  p.bits = bits;
   for (int i = 0; i < count; ++i) {
-    if (pr[i].K % 64 != 0) return BITNET_ERR_UNSUPPORTED;
-    total += pr[i].N * pr[i].K / 4;
-    max_rowb = std::max<int64_t>(max_rowb, pr[i].K / 4);
+    if (pr[i].K % (64 * (3 - bits)) != 0) return BITNET_ERR_UNSUPPORTED;   // 16-byte packed rows
+    total += pr[i].N * (pr[i].K / 8 * bits);
+    max_rowb = std::max<int64_t>(max_rowb, pr[i].K / 8 * bits);
     Kmax = std::max<int64_t>(Kmax, pr[i].K);
     xmax = std::max<int64_t>(xmax, M * pr[i].K * esz);
   }
@@ -293,7 +294,8 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
   p.Kp_max = static_cast<int>(Kmax);
   // single-token activations are stored block-permuted for the lane-group
   // tasks; pre-quantised codes are copied as they are (warp tasks)
-  p.blocked = (pl.MT == 1 && !prequant) ? 1 : 0;
+  p.blocked = (pl.MT == 1 && !prequant) ? (bits == 2 ? 1 : 2) : 0;
+  if (bits == 1 && p.blocked != 2) return BITNET_ERR_UNSUPPORTED;   // 1-bit GEMV: one token, raw x
   (void)xmax;
   // Shapes, most preferred first: (activation buffers, slots per warp, budget).
   // Two activation buffers let the activation warp run a segment ahead.
@@ -335,7 +337,7 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
     g.resid = pr[i].resid;
     g.K = static_cast<int>(pr[i].K);
     g.N = static_cast<int>(pr[i].N);
-    const int64_t rowb = pr[i].K / 4;
+    const int64_t rowb = pr[i].K / 8 * bits;
     int64_t rc = slot / rowb;
     // a short stream: about one chunk per consumer warp
     if (!big) rc = std::min<int64_t>(rc, ((per_cta + rowb - 1) / rowb + kGsCW - 1) / kGsCW);
@@ -346,6 +348,7 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
       task = rc >= 8 ? kGsTaskG8R2 : (rc >= 4 ? kGsTaskG16R2 : (rc >= 2 ? kGsTaskG16R1 : kGsTaskG32R1));
       const int64_t unit = task == kGsTaskG8R2 ? 8 : (task == kGsTaskG16R2 ? 4 : (task == kGsTaskG16R1 ? 2 : 1));
       rc -= rc % unit;
+      if (bits == 1) task += kGsTaskB1;
     } else {
       task = kGsTaskWarp;
       const int64_t unit = pl.MT == 1 ? 4 : (pl.MT == 2 ? 2 : 1);
@@ -385,7 +388,7 @@ constexpr int kStreamMaxP = 256;
 // ---------------------------------------------------------------------------
 // Tensor-core GEMM launch.
 // ---------------------------------------------------------------------------
-template <int BM, int SS, int AS>
+template <int BM, int SS, int AS, int BITS>
 cudaError_t run_tc_t(const int8_t* xq, const TcParams& p, cudaStream_t st) {
   CUtensorMap map;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.K), static_cast<cuuint64_t>(p.M)};
@@ -396,7 +399,7 @@ cudaError_t run_tc_t(const int8_t* xq, const TcParams& p, cudaStream_t st) {
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto k = tc_gemm_kernel<BM, SS, AS>;
+  auto k = tc_gemm_kernel<BM, SS, AS, BITS>;
   constexpr int smem = tc_smem_bytes<BM, SS>();
   cudaError_t e = allow_smem(k, smem);
   if (e != cudaSuccess) return e;
@@ -407,7 +410,7 @@ cudaError_t run_tc_t(const int8_t* xq, const TcParams& p, cudaStream_t st) {
 // Persistent tiles of 256 weight rows x BM tokens, one CTA per SM (the
 // shared-memory request keeps a second CTA off the SM: both want all 512
 // TMEM columns).
-template <int BM, int SS, int AS>
+template <int BM, int SS, int AS, int BITS>
 cudaError_t run_tp_t(const int8_t* xq, const TcParams& p, int sms, cudaStream_t st) {
   static_assert(2 * tp_smem_bytes<BM, SS, AS>() > 233472, "one CTA per SM");
   CUtensorMap map;
@@ -419,7 +422,7 @@ cudaError_t run_tp_t(const int8_t* xq, const TcParams& p, int sms, cudaStream_t 
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto k = tc_gemm_persistent_kernel<BM, SS, AS>;
+  auto k = tc_gemm_persistent_kernel<BM, SS, AS, BITS>;
   constexpr int smem = tp_smem_bytes<BM, SS, AS>();
   cudaError_t e = allow_smem(k, smem);
   if (e != cudaSuccess) return e;
@@ -431,11 +434,16 @@ cudaError_t run_tp_t(const int8_t* xq, const TcParams& p, int sms, cudaStream_t 
 // Token tile BM = MMA N.  Up to 64 tokens: one CTA per 128-row tile, 4 TMEM
 // A buffers, at most 256 TMEM columns, so two CTAs can share an SM.  Beyond:
 // the persistent kernel.
-cudaError_t run_tc(const int8_t* xq, const TcParams& p, int sms, cudaStream_t st) {
-  if (p.M <= 16) return run_tc_t<16, 8, 4>(xq, p, st);
-  if (p.M <= 32) return run_tc_t<32, 8, 4>(xq, p, st);
-  if (p.M <= 64) return run_tc_t<64, 8, 4>(xq, p, st);
-  return run_tp_t<128, 6, 4>(xq, p, sms, st);
+template <int BITS>
+cudaError_t run_tc_bits(const int8_t* xq, const TcParams& p, int sms, cudaStream_t st) {
+  if (p.M <= 16) return run_tc_t<16, 8, 4, BITS>(xq, p, st);
+  if (p.M <= 32) return run_tc_t<32, 8, 4, BITS>(xq, p, st);
+  if (p.M <= 64) return run_tc_t<64, 8, 4, BITS>(xq, p, st);
+  return run_tp_t<128, 6, 4, BITS>(xq, p, sms, st);
+}
+
+cudaError_t run_tc(const int8_t* xq, const TcParams& p, int sms, cudaStream_t st, int bits = 2) {
+  return bits == 1 ? run_tc_bits<1>(xq, p, sms, st) : run_tc_bits<2>(xq, p, sms, st);
 }
 
 bitnet_status launch_result(cudaError_t e) {
@@ -554,6 +562,48 @@ bitnet_status bitnet_quant_weights(const float* W, int64_t N, int64_t K, float e
   return launch_result(cudaSuccess);
 }
 
+bitnet_status bitnet_quant_weights_b1(const float* W, int64_t N, int64_t K, int8_t* Wb, float* beta, void* ws,
+                                      size_t ws_bytes, bitnet_stream_t stream) {
+  // beta is the absmean of bitnet_quant_weights (same exact sum, same
+  // workspace); the signs replace the ternarisation.
+  bitnet_status s = bitnet_quant_weights(W, N, K, 0.0f, nullptr, beta, ws, ws_bytes, stream);
+  if (s != BITNET_OK || Wb == nullptr) return s;
+  if (!aligned16(Wb)) return BITNET_ERR_ALIGN;
+  DeviceInfo* d;
+  s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  const int64_t n = N * K;
+  binarise_kernel<<<elementwise_grid(n / 4, d), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(W, n / 4, Wb);
+  return launch_result(cudaSuccess);
+}
+
+bitnet_status bitnet_pack_b1(const int8_t* Wb, int64_t N, int64_t K, uint8_t* Wp, uint32_t* n_invalid,
+                             bitnet_stream_t stream) {
+  if (Wb == nullptr || Wp == nullptr) return BITNET_ERR_NULL;
+  if (check_shape(1, K, N) != BITNET_OK || K % 32 != 0) return BITNET_ERR_SHAPE;
+  if (!aligned16(Wb) || !aligned16(Wp)) return BITNET_ERR_ALIGN;
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  const int64_t groups = N * K / 32;
+  pack_b1_kernel<<<elementwise_grid(groups, d), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      Wb, groups, reinterpret_cast<uint32_t*>(Wp), n_invalid);
+  return launch_result(cudaSuccess);
+}
+
+bitnet_status bitnet_unpack_b1(const uint8_t* Wp, int64_t N, int64_t K, int8_t* Wb, bitnet_stream_t stream) {
+  if (Wb == nullptr || Wp == nullptr) return BITNET_ERR_NULL;
+  if (check_shape(1, K, N) != BITNET_OK || K % 32 != 0) return BITNET_ERR_SHAPE;
+  if (!aligned16(Wb) || !aligned16(Wp)) return BITNET_ERR_ALIGN;
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  const int64_t groups = N * K / 32;
+  unpack_b1_kernel<<<elementwise_grid(groups, d), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint32_t*>(Wp), groups, Wb);
+  return launch_result(cudaSuccess);
+}
+
 bitnet_status bitnet_ternarise(const float* W, int64_t N, int64_t K, const float* gamma, float eps, int8_t* Wq,
                                bitnet_stream_t stream) {
   if (W == nullptr || gamma == nullptr || Wq == nullptr) return BITNET_ERR_NULL;
@@ -633,7 +683,7 @@ static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in
                                  const int32_t* sum_in, int64_t M, int64_t K, const uint8_t* Wp, int64_t N,
                                  const float* gamma, const float* rms_gain, float rms_eps, void* y, int y_dtype,
                                  int32_t* acc, void* ws, size_t ws_bytes, int path, cudaStream_t st,
-                                 const void* x2 = nullptr, const void* resid = nullptr) {
+                                 const void* x2 = nullptr, const void* resid = nullptr, int bits = 2) {
   if (Wp == nullptr || gamma == nullptr || ws == nullptr) return BITNET_ERR_NULL;
   if (y == nullptr && acc == nullptr) return BITNET_ERR_NULL;
   if (resid != nullptr && y == nullptr) return BITNET_ERR_NULL;
@@ -657,6 +707,11 @@ static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in
   // the gated input and the residual are in the streaming GEMV (K % 64 == 0)
   // and the tensor-core path, not in the padded-row GEMV
   if ((x2 != nullptr || resid != nullptr) && K % 64 != 0) gemv_ok = false;
+  // 1-bit signs: the streaming GEMV for one token, the tensor-core path otherwise
+  if (bits == 1) {
+    if (K % 128 != 0) return BITNET_ERR_SHAPE;
+    gemv_ok = (M == 1 && x != nullptr);
+  }
   if (path == BITNET_PATH_GEMV && !gemv_ok) return BITNET_ERR_UNSUPPORTED;
   const bool use_gemv = (path == BITNET_PATH_GEMV) || (path == BITNET_PATH_AUTO && gemv_ok);
 
@@ -666,7 +721,7 @@ static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in
     auto* pl = new (std::nothrow) StreamPlan<kStreamSmallP>;
     if (pl == nullptr) return BITNET_ERR_CUDA;
     s = plan_stream<kStreamSmallP>(d, &sp, 1, M, x != nullptr ? x_dtype : BITNET_F32, x == nullptr, rms_eps,
-                                   y != nullptr ? y_dtype : BITNET_F32, *pl);
+                                   y != nullptr ? y_dtype : BITNET_F32, *pl, bits);
     if (s == BITNET_OK) {
       pl->p.limit_ns = limit;
       pl->p.status = status;
@@ -734,7 +789,7 @@ static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in
   p.wvec = (K % 64 == 0) ? 1 : 0;
   p.limit_ns = limit;
   p.status = status;
-  return launch_result(run_tc(xq, p, d->sms, st));
+  return launch_result(run_tc(xq, p, d->sms, st, bits));
 }
 
 bitnet_status bitnet_linear_ex(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t* Wp, int64_t N,
@@ -765,6 +820,17 @@ bitnet_status bitnet_linear_relu2(const void* gate, const void* up, int x_dtype,
                      nullptr, ws, ws_bytes, BITNET_PATH_AUTO, reinterpret_cast<cudaStream_t>(stream), up, resid);
 }
 
+bitnet_status bitnet_linear_b1(const void* x, int x_dtype, int64_t M, int64_t K, const uint8_t* Wp, int64_t N,
+                               const float* beta, const float* rms_gain, float rms_eps, void* y, int y_dtype,
+                               void* ws, size_t ws_bytes, bitnet_stream_t stream) {
+  if (x == nullptr || y == nullptr) return BITNET_ERR_NULL;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (!aligned16(x)) return BITNET_ERR_ALIGN;
+  return linear_impl(x, x_dtype, nullptr, nullptr, nullptr, M, K, Wp, N, beta, rms_gain, rms_eps, y, y_dtype,
+                     nullptr, ws, ws_bytes, BITNET_PATH_AUTO, reinterpret_cast<cudaStream_t>(stream), nullptr,
+                     nullptr, 1);
+}
+
 bitnet_status bitnet_linear_q(const int8_t* xq, const float* x_scale, const int32_t* x_sum, int64_t M, int64_t K,
                               const uint8_t* Wp, int64_t N, const float* gamma, void* y, int y_dtype, int32_t* acc,
                               void* ws, size_t ws_bytes, int path, bitnet_stream_t stream) {
@@ -774,13 +840,14 @@ bitnet_status bitnet_linear_q(const int8_t* xq, const float* x_scale, const int3
                      ws_bytes, path, reinterpret_cast<cudaStream_t>(stream));
 }
 
-bitnet_status bitnet_linear_grouped(const bitnet_gemv_problem* problems, int count, int64_t M, int x_dtype,
-                                    float rms_eps, int y_dtype, void* ws, size_t ws_bytes, bitnet_stream_t stream) {
+static bitnet_status grouped_impl(const bitnet_gemv_problem* problems, int count, int64_t M, int x_dtype,
+                                  float rms_eps, int y_dtype, void* ws, size_t ws_bytes, bitnet_stream_t stream,
+                                  int bits) {
   if (problems == nullptr || ws == nullptr) return BITNET_ERR_NULL;
   if (count < 1 || count > kStreamMaxP) return BITNET_ERR_SHAPE;
   if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
   if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
-  if (M < 1 || M > kGemvMaxM) return BITNET_ERR_SHAPE;
+  if (M < 1 || M > (bits == 1 ? 1 : kGemvMaxM)) return BITNET_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < kWsHeader) return BITNET_ERR_WORKSPACE;
   std::vector<StreamProblem> sp(count);
   for (int i = 0; i < count; ++i) {
@@ -788,7 +855,7 @@ bitnet_status bitnet_linear_grouped(const bitnet_gemv_problem* problems, int cou
     if (q.x == nullptr || q.Wp == nullptr || q.gamma == nullptr || q.y == nullptr) return BITNET_ERR_NULL;
     bitnet_status s = check_shape(M, q.K, q.N);
     if (s != BITNET_OK) return s;
-    if (q.K % 64 != 0) return BITNET_ERR_SHAPE;
+    if (q.K % (64 * (3 - bits)) != 0) return BITNET_ERR_SHAPE;
     if (!aligned16(q.x) || !aligned16(q.Wp) || !aligned16(q.y) || (q.rms_gain != nullptr && !aligned16(q.rms_gain)))
       return BITNET_ERR_ALIGN;
     sp[i] = StreamProblem{q.x, q.Wp, q.gamma, q.rms_gain, nullptr, q.y, nullptr, q.K, q.N};
@@ -801,7 +868,7 @@ bitnet_status bitnet_linear_grouped(const bitnet_gemv_problem* problems, int cou
   if (count <= kStreamSmallP) {
     auto* pl = new (std::nothrow) StreamPlan<kStreamSmallP>;
     if (pl == nullptr) return BITNET_ERR_CUDA;
-    s = plan_stream<kStreamSmallP>(d, sp.data(), count, M, x_dtype, false, rms_eps, y_dtype, *pl);
+    s = plan_stream<kStreamSmallP>(d, sp.data(), count, M, x_dtype, false, rms_eps, y_dtype, *pl, bits);
     cudaError_t e = cudaSuccess;
     if (s == BITNET_OK) {
       pl->p.limit_ns = limit;
@@ -813,7 +880,7 @@ bitnet_status bitnet_linear_grouped(const bitnet_gemv_problem* problems, int cou
   }
   auto* pl = new (std::nothrow) StreamPlan<kStreamMaxP>;
   if (pl == nullptr) return BITNET_ERR_CUDA;
-  s = plan_stream<kStreamMaxP>(d, sp.data(), count, M, x_dtype, false, rms_eps, y_dtype, *pl);
+  s = plan_stream<kStreamMaxP>(d, sp.data(), count, M, x_dtype, false, rms_eps, y_dtype, *pl, bits);
   cudaError_t e = cudaSuccess;
   if (s == BITNET_OK) {
     pl->p.limit_ns = limit;
@@ -822,6 +889,16 @@ bitnet_status bitnet_linear_grouped(const bitnet_gemv_problem* problems, int cou
   }
   delete pl;
   return s != BITNET_OK ? s : launch_result(e);
+}
+
+bitnet_status bitnet_linear_grouped(const bitnet_gemv_problem* problems, int count, int64_t M, int x_dtype,
+                                    float rms_eps, int y_dtype, void* ws, size_t ws_bytes, bitnet_stream_t stream) {
+  return grouped_impl(problems, count, M, x_dtype, rms_eps, y_dtype, ws, ws_bytes, stream, 2);
+}
+
+bitnet_status bitnet_linear_grouped_b1(const bitnet_gemv_problem* problems, int count, int x_dtype, float rms_eps,
+                                       int y_dtype, void* ws, size_t ws_bytes, bitnet_stream_t stream) {
+  return grouped_impl(problems, count, 1, x_dtype, rms_eps, y_dtype, ws, ws_bytes, stream, 1);
 }
 
 bitnet_status bitnet_watchdog_selftest(void* ws, size_t ws_bytes, uint32_t limit_us, bitnet_stream_t stream) {

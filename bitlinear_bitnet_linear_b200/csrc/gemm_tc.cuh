@@ -62,32 +62,58 @@ __host__ __device__ constexpr int tc_smem_bytes() {
   return 1024 /* alignment slack */ + SS * BM * kTcBK + 512 /* barriers, flags */;
 }
 
-// Read the packed codes of one weight row for K block kb (32 bytes = 128
-// weights) into 8 words; bytes past the row end (or rows past N) read as 0.
+// Read the packed codes of one weight row for K block kb (128 weights: 32
+// bytes of 2-bit codes, or 16 bytes of 1-bit signs) into words w[0 .. 4 BITS);
+// bytes past the row end (or rows past N) read as 0.
+template <int BITS>
 __device__ __forceinline__ void tc_load_row_block(const uint8_t* __restrict__ row, bool valid, int rowbytes,
                                                   int kb, int wvec, uint32_t (&w)[8]) {
 #pragma unroll
   for (int i = 0; i < 8; ++i) w[i] = 0u;
   if (!valid) return;
-  const int off = kb * 32;
+  const int off = kb * 16 * BITS;
   const int avail = rowbytes - off;   // > 0, multiple of 4 (16 when wvec)
   if (wvec) {
     const uint4* p = reinterpret_cast<const uint4*>(row + off);
     const uint4 a = __ldg(p);
     w[0] = a.x; w[1] = a.y; w[2] = a.z; w[3] = a.w;
-    if (avail >= 32) {
+    if (BITS == 2 && avail >= 32) {
       const uint4 b = __ldg(p + 1);
       w[4] = b.x; w[5] = b.y; w[6] = b.z; w[7] = b.w;
     }
   } else {
     const uint32_t* p = reinterpret_cast<const uint32_t*>(row + off);
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 4 * BITS; ++i)
       if (4 * i < avail) w[i] = __ldg(p + i);
   }
 }
 
-template <int BM, int SS, int AS>
+// The 16 unsigned bytes (one per weight, weights 16c .. 16c + 15 of the K
+// block) of 16-byte chunk c, from the words of tc_load_row_block.  2-bit:
+// field s of word c holds weights 16c + 4s .. + 3 (code c = q + 1).  1-bit:
+// word c/2 holds weights 32(c/2) + 4s + j at bit 8j + s; chunk c takes
+// s = 4(c % 2) .. + 3 (bit 1 for +1).
+template <int BITS>
+__device__ __forceinline__ uint4 tc_expand_chunk(const uint32_t (&w)[8], int c) {
+  if constexpr (BITS == 2) {
+    const uint32_t v = w[c];
+    return make_uint4(v & 0x03030303u, (v >> 2) & 0x03030303u, (v >> 4) & 0x03030303u, (v >> 6) & 0x03030303u);
+  } else {
+    const uint32_t v = w[c >> 1] >> (4 * (c & 1));
+    return make_uint4(v & 0x01010101u, (v >> 1) & 0x01010101u, (v >> 2) & 0x01010101u, (v >> 3) & 0x01010101u);
+  }
+}
+
+// The exact dot product from the unsigned-code accumulator v and the code
+// sum: 2-bit codes c = q + 1 give v - sum x; 1-bit signs b = (q + 1) / 2
+// give 2 v - sum x.
+template <int BITS>
+__device__ __forceinline__ int tc_dot(uint32_t v, int xsum) {
+  return BITS == 2 ? static_cast<int>(v) - xsum : 2 * static_cast<int>(v) - xsum;
+}
+
+template <int BM, int SS, int AS, int BITS = 2>
 __global__ void __launch_bounds__(kTcThreads, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
   static_assert(BM % 16 == 0 && BM >= 16 && BM <= 256, "MMA N must be a multiple of 16 in [16, 256]");
@@ -198,14 +224,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int row = q * 32 + lane;
     const int n = n0 + row;
     const bool valid = n < p.N;
-    const int rowbytes = p.K / 4;
+    const int rowbytes = p.K * BITS / 8;
     const uint8_t* wrow = p.Wp + static_cast<int64_t>(valid ? n : 0) * rowbytes;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
 
     uint32_t wb[kPD][8];
 #pragma unroll
     for (int j = 0; j < kPD; ++j)
-      if (j < KB) tc_load_row_block(wrow, valid, rowbytes, j, p.wvec, wb[j]);
+      if (j < KB) tc_load_row_block<BITS>(wrow, valid, rowbytes, j, p.wvec, wb[j]);
 
     bool ok = true;
     for (int kb0 = 0; kb0 < KB && ok; kb0 += kPD) {
@@ -225,17 +251,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             uint32_t codes[32];
 #pragma unroll
             for (int g = 0; g < 8; ++g) {
-              const uint32_t w = wb[j][g];
-              codes[4 * g + 0] = w & 0x03030303u;
-              codes[4 * g + 1] = (w >> 2) & 0x03030303u;
-              codes[4 * g + 2] = (w >> 4) & 0x03030303u;
-              codes[4 * g + 3] = (w >> 6) & 0x03030303u;
+              const uint4 c4 = tc_expand_chunk<BITS>(wb[j], g);
+              codes[4 * g + 0] = c4.x;
+              codes[4 * g + 1] = c4.y;
+              codes[4 * g + 2] = c4.z;
+              codes[4 * g + 3] = c4.w;
             }
             tmem_st_32x32b_x32(tmem + lane_base + kACol0 + 32u * a, codes);
             tc_wait_st();
             tc_fence_before();
             mbar_arrive(&afull[a]);
-            if (kb + kPD < KB) tc_load_row_block(wrow, valid, rowbytes, kb + kPD, p.wvec, wb[j]);
+            if (kb + kPD < KB) tc_load_row_block<BITS>(wrow, valid, rowbytes, kb + kPD, p.wvec, wb[j]);
           } else {
             ok = false;
           }
@@ -271,7 +297,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int xsi = __shfl_sync(0xffffffffu, xsum, i);
           const int m = m0 + c0 + i;
           if (valid && m < p.M) {
-            const int a = static_cast<int>(v[i]) - xsi;
+            const int a = tc_dot<BITS>(v[i], xsi);
             const int64_t idx = static_cast<int64_t>(m) * p.N + n;
             if (p.acc != nullptr) p.acc[idx] = a;
             if (p.y != nullptr) {
@@ -328,7 +354,7 @@ __host__ __device__ constexpr int tp_smem_bytes() {
   return 1024 /* alignment slack */ + SS * BM * kTcBK + AS * kTpAStage + 1024 /* barriers, flags */;
 }
 
-template <int BM, int SS, int AS>
+template <int BM, int SS, int AS, int BITS = 2>
 __global__ void __launch_bounds__(kTpThreads, 1)
     tc_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
   static_assert(BM == 128, "two buffers of 2 x BM accumulator columns fill TMEM");
@@ -468,14 +494,15 @@ __global__ void __launch_bounds__(kTpThreads, 1)
   } else if (warp < 10) {
     // ------------------------------------------------------------ converters
     const int row = (warp - 2) * 32 + lane;          // A row of the 256-row tile
-    const int rowbytes = p.K / 4;
+    const int rowbytes = p.K * BITS / 8;
     const int total = my_tiles * KB;
     uint32_t wb[kPD][8];
     auto load = [&](int gi, uint32_t (&w)[8]) {
       const int i = gi / KB, kb = gi - i * KB;
       const int n = tile_n0(i) + row;
       const bool valid = n < p.N;
-      tc_load_row_block(p.Wp + static_cast<int64_t>(valid ? n : 0) * rowbytes, valid, rowbytes, kb, p.wvec, w);
+      tc_load_row_block<BITS>(p.Wp + static_cast<int64_t>(valid ? n : 0) * rowbytes, valid, rowbytes, kb, p.wvec,
+                              w);
     };
 #pragma unroll
     for (int j = 0; j < kPD; ++j)
@@ -495,13 +522,9 @@ __global__ void __launch_bounds__(kTpThreads, 1)
           } else {
             uint8_t* arow = as + a * kTpAStage + row * kTcBK;
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-              // word c covers weights 16c .. 16c + 15: field s holds 16c + 4s .. + 3
-              const uint32_t w = wb[j][c];
+            for (int c = 0; c < 8; ++c)   // chunk c: weights 16c .. 16c + 15 of the K block
               *reinterpret_cast<uint4*>(arow + ((static_cast<uint32_t>(c) ^ swz) << 4)) =
-                  make_uint4(w & 0x03030303u, (w >> 2) & 0x03030303u, (w >> 4) & 0x03030303u,
-                             (w >> 6) & 0x03030303u);
-            }
+                  tc_expand_chunk<BITS>(wb[j], c);
             // the tensor core reads these bytes through the async proxy
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             mbar_arrive(&afull[a]);
@@ -576,7 +599,7 @@ __global__ void __launch_bounds__(kTpThreads, 1)
             const int xst = __shfl_sync(0xffffffffu, xsc_, t);
             if (valid && m0 + 32 * c + t < p.M)
               yb[static_cast<int64_t>(t) * p.N] =
-                  bf16_bits_rne(__fmul_rn(small_int_to_float(static_cast<int>(v[t]) - xst), gst));
+                  bf16_bits_rne(__fmul_rn(small_int_to_float(tc_dot<BITS>(v[t], xst)), gst));
           }
         } else {
 #pragma unroll
@@ -585,7 +608,7 @@ __global__ void __launch_bounds__(kTpThreads, 1)
             const int xst = __shfl_sync(0xffffffffu, xsc_, t);
             const int m = m0 + 32 * c + t;
             if (valid && m < p.M) {
-              const int acc = static_cast<int>(v[t]) - xst;
+              const int acc = tc_dot<BITS>(v[t], xst);
               const int64_t idx = static_cast<int64_t>(m) * p.N + n;
               if (p.acc != nullptr) p.acc[idx] = acc;
               if (p.y != nullptr) {

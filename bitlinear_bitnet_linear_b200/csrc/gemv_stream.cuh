@@ -51,6 +51,7 @@ constexpr int kGsTaskG16R2 = 1;     // 4-row tasks
 constexpr int kGsTaskG16R1 = 2;     // 2-row tasks
 constexpr int kGsTaskG32R1 = 3;     // 1-row tasks
 constexpr int kGsTaskWarp = 4;      // whole warp over R = 4 / 2 / 1 rows (M = 1 / 2 / 4), linear codes
+constexpr int kGsTaskB1 = 5;        // 1-bit signs: kGsTaskB1 + (a G/RS shape above, 0 .. 3)
 
 struct GsProblem {
   const void* x;          // [M, K] raw activations (x_dtype) or int8 codes (prequant)
@@ -77,7 +78,8 @@ struct GsParams {
   int64_t total_bytes;
   int slot_bytes, nslots;        // ring of each consumer warp
   int nxb;                       // activation code buffers (2: quantise a segment ahead)
-  int blocked;                   // 1: codes in the block-permuted layout (lane-group tasks)
+  int blocked;                   // 1 / 2: codes block-permuted in 4 / 8 quarters (lane-group tasks)
+  int bits;                      // 2: ternary codes, 2 bits per weight; 1: BitNet b1 signs
   int Kp_max;                    // int8 code rows in shared memory (K rounded up to 64)
   uint64_t limit_ns;
   uint32_t* status;
@@ -103,7 +105,7 @@ __device__ __forceinline__ void gs_cta_start(const GsParams<MAXP>& p, int b, int
   int lo = 0, hi = p.nprob;   // first problem whose bytes end after target
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
-    const int64_t end = p.prob[mid].byte0 + static_cast<int64_t>(p.prob[mid].K / 4) * p.prob[mid].N;
+    const int64_t end = p.prob[mid].byte0 + static_cast<int64_t>(p.prob[mid].K / 8 * p.bits) * p.prob[mid].N;
     if (target < end)
       hi = mid;
     else
@@ -112,7 +114,7 @@ __device__ __forceinline__ void gs_cta_start(const GsParams<MAXP>& p, int b, int
   prob = lo;
   row = 0;
   if (lo == p.nprob) return;
-  const int64_t rb = p.prob[lo].K / 4;
+  const int64_t rb = p.prob[lo].K / 8 * p.bits;
   // target may sit inside the previous problem's last row (before byte0)
   const int64_t off = target > p.prob[lo].byte0 ? target - p.prob[lo].byte0 : 0;
   const int64_t r = (off + rb - 1) / rb;
@@ -204,6 +206,92 @@ __device__ __forceinline__ void gs_task_lg(const uint8_t* wbase, int rc, int row
     if (lj == i && i < nr) {
       const int64_t n = r + rb + i;
       const int accv = a[i][0] - xsum0;
+      if (P.acc != nullptr) P.acc[n] = accv;
+      if (P.y != nullptr) {
+        float o = __fmul_rn(__int2float_rn(accv), gs0);
+        if (P.resid != nullptr) o = __fadd_rn(load_y(P.resid, y_dtype, n), o);
+        store_y(P.y, y_dtype, n, o);
+      }
+    }
+  }
+}
+
+// BitNet b1 signs, M = 1: as gs_task_lg, with 16 bytes of packed signs per
+// row per step (128 weights, chunk c) against eight 16-byte activation
+// blocks (xs_blocked8).  Word e of the chunk holds weights 32e + 4s + j at
+// bit 8j + s; masking field s (0x01010101 << s) lines four signs (scaled by
+// 2^s) up with four activations; eight per-field accumulators are rescaled
+// by exact shifts.  With signs b = (q + 1) / 2: sum q x = 2 sum b x - sum x.
+template <int G, int RS>
+__device__ __forceinline__ void gs_task_lg_b1(const uint8_t* wbase, int rc, int row0, int rowb, int nchunk,
+                                              const int8_t* xs, int lane, int xsum0, float gs0, const GsProblem& P,
+                                              int r, int y_dtype) {
+  const int lg = lane / G, lj = lane % G;
+  const int rb = row0 + lg * RS;
+  const int nr = max(0, min(RS, rc - rb));
+  const int xq8 = rowb;                          // K / 8: distance between the eight block quarters
+  int a[RS][8];
+#pragma unroll
+  for (int i = 0; i < RS; ++i)
+#pragma unroll
+    for (int f = 0; f < 8; ++f) a[i][f] = 0;
+  auto body = [&](const uint4 (&w)[RS], const int8_t* xp) {
+    uint4 xv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) xv[e] = *reinterpret_cast<const uint4*>(xp + e * xq8);
+#pragma unroll
+    for (int i = 0; i < RS; ++i) {
+      const uint32_t wv[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint4 lo = xv[2 * e], hi = xv[2 * e + 1];
+        a[i][0] = dp4a_us(wv[e] & 0x01010101u, lo.x, a[i][0]);
+        a[i][1] = dp4a_us(wv[e] & 0x02020202u, lo.y, a[i][1]);
+        a[i][2] = dp4a_us(wv[e] & 0x04040404u, lo.z, a[i][2]);
+        a[i][3] = dp4a_us(wv[e] & 0x08080808u, lo.w, a[i][3]);
+        a[i][4] = dp4a_us(wv[e] & 0x10101010u, hi.x, a[i][4]);
+        a[i][5] = dp4a_us(wv[e] & 0x20202020u, hi.y, a[i][5]);
+        a[i][6] = dp4a_us(wv[e] & 0x40404040u, hi.z, a[i][6]);
+        a[i][7] = dp4a_us(wv[e] & 0x80808080u, hi.w, a[i][7]);
+      }
+    }
+  };
+  const uint8_t* wrow = wbase + static_cast<int64_t>(rb) * rowb + 16 * lj;
+  const int8_t* xp = xs + 16 * lj;
+  if (nr == RS) {
+    for (int c = lj; c < nchunk; c += G) {
+      uint4 w[RS];
+#pragma unroll
+      for (int i = 0; i < RS; ++i) w[i] = *reinterpret_cast<const uint4*>(wrow + i * rowb);
+      body(w, xp);
+      wrow += 16 * G;
+      xp += 16 * G;
+    }
+  } else if (nr > 0) {
+    for (int c = lj; c < nchunk; c += G) {
+      uint4 w[RS];
+#pragma unroll
+      for (int i = 0; i < RS; ++i)
+        w[i] = (i < nr) ? *reinterpret_cast<const uint4*>(wrow + i * rowb) : make_uint4(0u, 0u, 0u, 0u);
+      body(w, xp);
+      wrow += 16 * G;
+      xp += 16 * G;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < RS; ++i) {
+    int t = 0;
+#pragma unroll
+    for (int f = 0; f < 8; ++f) t += a[i][f] >> f;
+#pragma unroll
+    for (int o = G / 2; o >= 1; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    a[i][0] = t;
+  }
+#pragma unroll
+  for (int i = 0; i < RS; ++i) {
+    if (lj == i && i < nr) {
+      const int64_t n = r + rb + i;
+      const int accv = 2 * a[i][0] - xsum0;
       if (P.acc != nullptr) P.acc[n] = accv;
       if (P.y != nullptr) {
         float o = __fmul_rn(__int2float_rn(accv), gs0);
@@ -354,7 +442,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
   uint8_t* myslots = wslots + static_cast<size_t>(warp) * p.nslots * p.slot_bytes;
   auto issue = [&](int slot) {
     const GsProblem& Q = p.prob[icur.q];
-    const int64_t rowb = Q.K / 4;
+    const int64_t rowb = Q.K / 8 * p.bits;
     const uint32_t bytes = static_cast<uint32_t>(min(Q.rc, icur.r1 - icur.r) * rowb);
     mbar_expect_tx(&H.wfull[warp][slot], bytes);
     bulk_g2s(myslots + slot * p.slot_bytes, Q.Wp + static_cast<int64_t>(icur.r) * rowb, bytes, &H.wfull[warp][slot]);
@@ -418,7 +506,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
       ok = copy_codes(P, xs, Kp, sc, &H.q.qpart[0][0], kAll, 0, tid == CW * 32) && ok;
     } else {
       quant_rows<kAll, MT, 1, false, kGsBarAll, false>(static_cast<const char*>(P.x), p.x_dtype, P.K * esz, p.M,
-                                                      P.K, P.gain, p.rms_eps, xs, Kp, H.q, sc, 0, p.blocked != 0,
+                                                      P.K, P.gain, p.rms_eps, xs, Kp, H.q, sc, 0, p.blocked,
                                                       static_cast<const char*>(P.x2));
     }
     group_sync<kGsBarAll, kAll>();
@@ -466,7 +554,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
       } else {
         quant_rows<32, MT, 1, false, kGsBarX, false>(static_cast<const char*>(P.x), p.x_dtype, P.K * esz, p.M,
                                                      P.K, P.gain, p.rms_eps, xs, Kp, H.qx, sc, CW * 32,
-                                                     p.blocked != 0, static_cast<const char*>(P.x2));
+                                                     p.blocked, static_cast<const char*>(P.x2));
       }
       __syncwarp();
       if (lane == 0) {
@@ -516,7 +604,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
     if (q < qlast) gamma_next = __ldg(p.prob[q + 1].gamma);   // in flight during this segment
     const float gs0 = __fmul_rn(gamma, sc[0]);
     const int nword = P.K / 16;      // 32-bit code words (16 weights) per row
-    const int rowb = P.K / 4, nchunk = P.K / 64;
+    const int rowb = P.K / 8 * p.bits, nchunk = P.K / (64 * (3 - p.bits));   // 16-byte chunks per row
     while (cur.q == q) {
       if (!gs_wait(&H.wfull[warp][slot], phase, p.limit_ns, abort_flag)) {
         ok = false;
@@ -537,6 +625,20 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
       } else if (MT == 1 && P.task == kGsTaskG32R1) {
         for (int row0 = 0; row0 < rows; ++row0)
           gs_task_lg<32, 1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+      } else if (MT == 1 && P.task >= kGsTaskB1) {
+        if (P.task == kGsTaskB1 + kGsTaskG8R2) {
+          for (int row0 = 0; row0 < rows; row0 += 8)
+            gs_task_lg_b1<8, 2>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+        } else if (P.task == kGsTaskB1 + kGsTaskG16R2) {
+          for (int row0 = 0; row0 < rows; row0 += 4)
+            gs_task_lg_b1<16, 2>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+        } else if (P.task == kGsTaskB1 + kGsTaskG16R1) {
+          for (int row0 = 0; row0 < rows; row0 += 2)
+            gs_task_lg_b1<16, 1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+        } else {
+          for (int row0 = 0; row0 < rows; ++row0)
+            gs_task_lg_b1<32, 1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+        }
       } else {
         constexpr int R = (MT == 1) ? 4 : ((MT == 2) ? 2 : 1);
         const uint32_t* wbase = reinterpret_cast<const uint32_t*>(wb8);

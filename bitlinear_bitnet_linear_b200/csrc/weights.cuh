@@ -241,6 +241,69 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint32_t* __restrict_
 // Empty kernel launched WITHOUT programmatic serialisation after calls that
 // write weights: a following GEMV may read weights before its dependency
 // wait, so the weight writer must be fully complete first.
+// BitNet b1 ("BitNet / Ternary / Binary", BitNet b1 (binaire): every weight
+// exactly +1 or -1): W_b = +1 where W >= 0, else -1 (NaN gives -1).
+__global__ void __launch_bounds__(256) binarise_kernel(const float* __restrict__ W, int64_t n4,
+                                                       int8_t* __restrict__ Wb) {
+  const float4* W4 = reinterpret_cast<const float4*>(W);
+  char4* B4 = reinterpret_cast<char4*>(Wb);
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4 v = __ldg(W4 + i);
+    char4 b;
+    b.x = v.x >= 0.0f ? 1 : -1;
+    b.y = v.y >= 0.0f ? 1 : -1;
+    b.z = v.z >= 0.0f ? 1 : -1;
+    b.w = v.w >= 0.0f ? 1 : -1;
+    B4[i] = b;
+  }
+}
+
+// 1-bit pack: one uint32 per 32 weights, weight 32g + 4s + j at bit 8j + s
+// (bit 1 for +1).  Values other than +-1 are stored as 0 and counted.
+__global__ void __launch_bounds__(256) pack_b1_kernel(const int8_t* __restrict__ Wb, int64_t ngroups,
+                                                      uint32_t* __restrict__ Wp, uint32_t* n_invalid) {
+  uint32_t bad = 0;
+  const uint4* Q = reinterpret_cast<const uint4*>(Wb);
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < ngroups;
+       g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint4 a = __ldg(Q + 2 * g), b = __ldg(Q + 2 * g + 1);
+    const uint32_t in[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};   // in[s] byte j = w[32g + 4s + j]
+    uint32_t word = 0;
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int v = static_cast<int8_t>((in[s] >> (8 * j)) & 0xffu);
+        if (v == 1)
+          word |= 1u << (8 * j + s);
+        else if (v != -1)
+          ++bad;
+      }
+    }
+    Wp[g] = word;
+  }
+  if (n_invalid != nullptr && bad) atomicAdd(n_invalid, bad);
+}
+
+__global__ void __launch_bounds__(256) unpack_b1_kernel(const uint32_t* __restrict__ Wp, int64_t ngroups,
+                                                        int8_t* __restrict__ Wb) {
+  uint4* Q = reinterpret_cast<uint4*>(Wb);
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < ngroups;
+       g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t word = __ldg(Wp + g);
+    uint32_t out[8];
+#pragma unroll
+    for (int s = 0; s < 8; ++s) {
+      // bits (word >> s) & 0x01010101 are the weights 32g + 4s .. + 3: 1 -> +1, 0 -> -1 (0xff)
+      const uint32_t bits = (word >> s) & 0x01010101u;
+      out[s] = bits | ((0x01010101u - bits) * 0xffu);
+    }
+    Q[2 * g] = make_uint4(out[0], out[1], out[2], out[3]);
+    Q[2 * g + 1] = make_uint4(out[4], out[5], out[6], out[7]);
+  }
+}
+
 __global__ void stream_fence_kernel() {}
 
 }  // namespace bitnet

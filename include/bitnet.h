@@ -143,6 +143,44 @@ bitnet_status bitnet_unpack(const uint8_t *Wp, int64_t N, int64_t K, int8_t *Wq,
                             uint32_t *n_invalid, bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * BitNet b1 binary weights ("BitNet / Ternary / Binary -- Les LLMs 1-bit",
+ * BitNet b1 (binaire): every weight of the BitLinear layer is exactly +1
+ * or -1).  The pages give no binarisation rule; this library reads it as
+ * the sign with ties to +1 and the absmean scale of the ternary case.
+ * ------------------------------------------------------------------------ */
+
+/* beta = mean|W| exactly as gamma in bitnet_quant_weights (same workspace
+ * and errors), and W_b = +1 where W >= 0, else -1 (NaN gives -1).
+ * Wb: [N, K] int8 output or NULL (beta only); beta: device binary32. */
+bitnet_status bitnet_quant_weights_b1(const float *W, int64_t N, int64_t K, int8_t *Wb,
+                                      float *beta, void *ws, size_t ws_bytes,
+                                      bitnet_stream_t stream);
+
+/* 1-bit pack: K % 32 == 0; group g of row n is the little-endian uint32 at
+ * byte n*K/8 + 4g; weight k = 32g + 4s + j (s in 0..7, j in 0..3) is bit
+ * 8j + s, 1 for +1 and 0 for -1.  Values other than +-1 are stored as 0
+ * and counted into *n_invalid (device uint32, may be NULL, accumulated).
+ * Wp: [N, K/8] uint8 output. */
+bitnet_status bitnet_pack_b1(const int8_t *Wb, int64_t N, int64_t K, uint8_t *Wp,
+                             uint32_t *n_invalid, bitnet_stream_t stream);
+
+/* Inverse of bitnet_pack_b1: every bit pattern is valid. */
+bitnet_status bitnet_unpack_b1(const uint8_t *Wp, int64_t N, int64_t K, int8_t *Wb,
+                               bitnet_stream_t stream);
+
+/* BitLinear forward with 1-bit weights: as bitnet_linear, with
+ *   acc[m,n] = sum_k x_q[m,k] * W_b[n,k] = 2 sum_{W_b = +1} x_q - sum_k x_q
+ *   y[m,n]   = (float)acc[m,n] * (beta * s_x[m]).
+ * K % 128 == 0 (else BITNET_ERR_SHAPE).  M = 1 runs the fused streaming
+ * GEMV; larger M the quantiser then the tensor-core GEMM.  Wp: [N, K/8]
+ * (bitnet_pack_b1).  ws: bitnet_workspace_bytes(M, K, N) bytes. */
+bitnet_status bitnet_linear_b1(const void *x, int x_dtype, int64_t M, int64_t K,
+                               const uint8_t *Wp, int64_t N, const float *beta,
+                               const float *rms_gain, float rms_eps,
+                               void *y, int y_dtype, void *ws, size_t ws_bytes,
+                               bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Per-call path.
  * ------------------------------------------------------------------------ */
 
@@ -275,6 +313,13 @@ bitnet_status bitnet_linear_grouped(const bitnet_gemv_problem *problems, int cou
  *   - Non-finite W is not reported (there is no workspace status word). */
 bitnet_status bitnet_quant_weights_noalloc(const float *W, int64_t N, int64_t K, float eps,
                                            int8_t *Wq, float *gamma, bitnet_stream_t stream);
+
+/* bitnet_linear_grouped for BitNet b1 weights (bitnet_pack_b1, Wp [N, K/8],
+ * gamma = beta), one token (M = 1), K % 128 == 0: each problem is computed
+ * exactly as bitnet_linear_b1. */
+bitnet_status bitnet_linear_grouped_b1(const bitnet_gemv_problem *problems, int count, int x_dtype,
+                                       float rms_eps, int y_dtype, void *ws, size_t ws_bytes,
+                                       bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * Failure detection.

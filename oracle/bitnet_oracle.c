@@ -341,6 +341,64 @@ void orc_unpack_b1(const uint8_t *Wp, int64_t N, int64_t K, int8_t *Wb)
 }
 
 /* ------------------------------------------------------------------------ */
+/* Base-3 packing ("BitNET Family", Memory Efficiency: 0.4 GB for the 2B     */
+/* model, i.e. about 1.6 bits per weight; Hacker News thread (bitsplea.se):  */
+/* "2 bits instead of 1.58").  Five ternary weights fit one byte            */
+/* (3^5 = 243 <= 256): a byte holds sum_i c_i 3^i with codes c = q + 1.     */
+/* Layout (this library's): K is cut into groups of 20 weights, one         */
+/* little-endian uint32 each; byte j of group g holds the weights           */
+/* k = 20g + 4i + j (i = 0..4, c_i the i-th base-3 digit), so digit i of the */
+/* four bytes gives four consecutive weights.  Weights past K code as 1     */
+/* (q = 0).  A row takes ceil(K / 80) * 16 bytes (whole 16-byte chunks).     */
+/* Values outside {-1, 0, 1} are stored as code 1 and counted.               */
+/* ------------------------------------------------------------------------ */
+int64_t orc_t3_row_bytes(int64_t K) { return (K + 79) / 80 * 16; }
+
+int64_t orc_pack_t3(const int8_t *Wq, int64_t N, int64_t K, uint8_t *Wp)
+{
+    int64_t bad = 0, rb = orc_t3_row_bytes(K);
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < rb / 4; ++g)
+            for (int j = 0; j < 4; ++j) {
+                int v = 0, p3 = 1;
+                for (int i = 0; i < 5; ++i) {
+                    int64_t k = 20 * g + 4 * i + j;
+                    int c = 1;
+                    if (k < K) {
+                        int q = Wq[n * K + k];
+                        if (q >= -1 && q <= 1) c = q + 1;
+                        else ++bad;
+                    }
+                    v += c * p3;
+                    p3 *= 3;
+                }
+                Wp[n * rb + 4 * g + j] = (uint8_t)v;
+            }
+    return bad;
+}
+
+/* Inverse of orc_pack_t3 for k < K; bytes above 242 are invalid: counted,  */
+/* their weights read as 0.                                                 */
+int64_t orc_unpack_t3(const uint8_t *Wp, int64_t N, int64_t K, int8_t *Wq)
+{
+    int64_t bad = 0, rb = orc_t3_row_bytes(K);
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < rb / 4; ++g)
+            for (int j = 0; j < 4; ++j) {
+                int v = Wp[n * rb + 4 * g + j];
+                int valid = v <= 242;
+                if (!valid && 20 * g + j < K) ++bad;
+                for (int i = 0; i < 5; ++i) {
+                    int64_t k = 20 * g + 4 * i + j;
+                    int c = v % 3;
+                    v /= 3;
+                    if (k < K) Wq[n * K + k] = valid ? (int8_t)(c - 1) : (int8_t)0;
+                }
+            }
+    return bad;
+}
+
+/* ------------------------------------------------------------------------ */
 /* ReLU^2 gate of the feed-forward layers.  [KeyTech] "Architectural        */
 /* Innovations": squared ReLU activations in the feed-forward layers.  The  */
 /* down projection's input is the gate projection's output squared after    */

@@ -62,6 +62,9 @@ def lib():
         L.orc_binarise.argtypes = [P, I64, P]; L.orc_binarise.restype = None
         L.orc_pack_b1.argtypes = [P, I64, I64, P]; L.orc_pack_b1.restype = I64
         L.orc_unpack_b1.argtypes = [P, I64, I64, P]; L.orc_unpack_b1.restype = None
+        L.orc_t3_row_bytes.argtypes = [I64]; L.orc_t3_row_bytes.restype = I64
+        L.orc_pack_t3.argtypes = [P, I64, I64, P]; L.orc_pack_t3.restype = I64
+        L.orc_unpack_t3.argtypes = [P, I64, I64, P]; L.orc_unpack_t3.restype = I64
         L.orc_output_resid.argtypes = [P, I64, I64, F, P, P, P]; L.orc_output_resid.restype = None
         _lib = L
     return _lib
@@ -186,6 +189,27 @@ def unpack_b1(Wp: np.ndarray, K: int) -> np.ndarray:
     out = np.empty((N, K), np.int8)
     lib().orc_unpack_b1(_p(Wp), N, K, _p(out))
     return out
+
+
+def t3_row_bytes(K: int) -> int:
+    return int(lib().orc_t3_row_bytes(K))
+
+
+def pack_t3(Wq: np.ndarray):
+    """Base-3, five weights per byte.  Returns (packed [N, t3_row_bytes(K)] uint8, n_invalid)."""
+    Wq = _c(Wq, np.int8)
+    N, K = Wq.shape
+    out = np.empty((N, t3_row_bytes(K)), np.uint8)
+    bad = lib().orc_pack_t3(_p(Wq), N, K, _p(out))
+    return out, int(bad)
+
+
+def unpack_t3(Wp: np.ndarray, K: int):
+    Wp = _c(Wp, np.uint8)
+    N = Wp.shape[0]
+    out = np.empty((N, K), np.int8)
+    bad = lib().orc_unpack_t3(_p(Wp), N, K, _p(out))
+    return out, int(bad)
 
 
 def relu2_gate(gate: np.ndarray, up: np.ndarray) -> np.ndarray:

@@ -463,3 +463,43 @@ def test_binary_contraction_add_subtract(orc):
     plus = (B == 1).astype(np.int64)
     assert np.array_equal(acc, x @ plus.T - x @ (1 - plus).T)
     assert np.array_equal(acc, 2 * (x @ plus.T) - x.sum(axis=1, keepdims=True))
+
+
+# ---------------------------------------------------------------------------
+# Base-3 packing (five ternary weights per byte, about 1.6 bits per weight:
+# "BitNET Family", Memory Efficiency; Hacker News, "2 bits instead of 1.58").
+# ---------------------------------------------------------------------------
+def test_pack_t3_golden(orc):
+    lines = golden_lines("pack_t3_layout.txt")
+    w = np.array([[int(v) for v in lines[0].split()]], np.int8)
+    want = np.array([[int(v, 16) for v in lines[1].split()]], np.uint8)
+    packed, bad = orc.pack_t3(w)
+    assert bad == 0 and np.array_equal(packed, want)
+
+
+@pytest.mark.parametrize("K", [16, 20, 80, 100, 2560, 6912])
+def test_pack_t3_roundtrip_and_size(orc, K):
+    rng = np.random.default_rng(K)
+    q = rng.integers(-1, 2, (7, K)).astype(np.int8)
+    P, bad = orc.pack_t3(q)
+    assert bad == 0 and P.shape == (7, (K + 79) // 80 * 16)
+    back, bad2 = orc.unpack_t3(P, K)
+    assert bad2 == 0 and np.array_equal(back, q)
+    assert P.max() <= 242
+    if K % 80 == 0:
+        assert P.shape[1] * 5 == K // 4 * 4        # 20% fewer bytes than 2 bits per weight
+
+
+def test_pack_t3_every_byte_value(orc):
+    """Each of the 243 byte values is one 5-digit base-3 word: digit i of byte j is weight 4i + j."""
+    for v in range(256):
+        P = np.full((1, 16), 121, np.uint8)          # 121 = every code 1 (weight 0)
+        P[0, 0] = v
+        w, bad = orc.unpack_t3(P, 80)
+        if v <= 242:
+            assert bad == 0
+            assert [int(w[0, 4 * i]) for i in range(5)] == [(v // 3 ** i) % 3 - 1 for i in range(5)]
+            assert orc.pack_t3(w)[0][0, 0] == v
+        else:
+            assert bad == 1 and all(w[0, 4 * i] == 0 for i in range(5))
+    assert orc.pack_t3(np.full((1, 20), 2, np.int8))[1] == 20      # out-of-range values counted

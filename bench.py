@@ -362,6 +362,36 @@ def run_ours(args):
                       f"{per_graph} steps"}
         del b1_graph, b1_call, b1_stack
 
+    # ---- base-3: the same ternary stack at five weights per byte ------------
+    t3 = None
+    if not args.no_chain:
+        t3_packed = []
+        with torch.cuda.stream(stream):
+            for (K, N, Wp, g) in stack:
+                t3_packed.append(bn.bitnet_pack_t3(bn.bitnet_unpack(Wp, K)))
+        torch.cuda.synchronize()
+        t3_call = bn.GroupedCall([(x, Wp3, g, gains[K], y) for (K, N, _, g), Wp3, x, y
+                                  in zip(stack, t3_packed, xs, ys)], rms_eps=1e-5, ws=ws, bits=3)
+
+        def t3_steps(n):
+            def fn():
+                for _ in range(n):
+                    t3_call()
+            return fn
+
+        t3_bytes = sum(N * bn.bitnet_t3_row_bytes(K) + K * 2 + N * 2 + 4 for (K, N, _, _) in stack)
+        t3_graph = capture(t3_steps(per_graph))
+        tsteps = (max(20, args.steps // 2) // per_graph) * per_graph
+        tms, tms_max, _ = time_graph(t3_graph, tsteps // per_graph, 3)
+        tms, tms_max = tms / per_graph, tms_max / per_graph
+        assert bn.bitnet_get_error(ws) == 0
+        t3 = {"value": round(world * t3_bytes / (tms_max * 1e-3) / 1e9, 2), "unit": "GB/s",
+              "ms_per_step": round(tms_max, 5), "tokens_per_s": round(world * 1e3 / tms_max, 1),
+              "bytes_per_step": t3_bytes, "steps": tsteps,
+              "what": "the same ternary stack packed base-3 (five weights per byte, 1.6 bits per weight), one "
+                      "grouped launch per token (bitnet_linear_grouped_t3), digits decoded in registers"}
+        del t3_graph, t3_call, t3_packed
+
     # ---- e2e: host buffers, through the public API, no graph ----------------
     e2e = None
     if not args.no_e2e:
@@ -460,6 +490,8 @@ def run_ours(args):
         out["ffn_chain"] = ffn
     if b1 is not None:
         out["b1_decode"] = b1
+    if t3 is not None:
+        out["t3_decode"] = t3
     if prefill is not None:
         out["prefill"] = prefill
     if cpu is not None:

@@ -28,7 +28,8 @@ EXPORTS = ("bitnet_workspace_bytes", "bitnet_quant_weights_workspace_bytes", "bi
            "bitnet_pack", "bitnet_unpack", "bitnet_quant_act", "bitnet_linear", "bitnet_linear_ex",
            "bitnet_linear_q", "bitnet_linear_grouped", "bitnet_linear_relu2", "bitnet_quant_act_relu2",
            "bitnet_quant_weights_b1", "bitnet_pack_b1", "bitnet_unpack_b1", "bitnet_linear_b1",
-           "bitnet_linear_grouped_b1",
+           "bitnet_linear_grouped_b1", "bitnet_t3_row_bytes", "bitnet_pack_t3", "bitnet_unpack_t3",
+           "bitnet_linear_t3", "bitnet_linear_grouped_t3",
            "bitnet_quant_weights_noalloc",
            "bitnet_set_wait_limit_us", "bitnet_watchdog_selftest")
 
@@ -77,6 +78,11 @@ def lib() -> ctypes.CDLL:
         "bitnet_unpack_b1": ([P, I64, I64, P, P], I32),
         "bitnet_linear_b1": ([P, I32, I64, I64, P, I64, P, P, F, P, I32, P, SZ, P], I32),
         "bitnet_linear_grouped_b1": ([P, I32, I32, F, I32, P, SZ, P], I32),
+        "bitnet_t3_row_bytes": ([I64], I64),
+        "bitnet_pack_t3": ([P, I64, I64, P, P, P], I32),
+        "bitnet_unpack_t3": ([P, I64, I64, P, P, P], I32),
+        "bitnet_linear_t3": ([P, I32, I64, P, I64, P, P, F, P, I32, P, SZ, P], I32),
+        "bitnet_linear_grouped_t3": ([P, I32, I32, F, I32, P, SZ, P], I32),
         "bitnet_linear_relu2": ([P, P, I32, I64, I64, P, I64, P, P, F, P, P, I32, P, SZ, P], I32),
         "bitnet_linear": ([P, I32, I64, I64, P, I64, P, P, F, P, I32, P, SZ, P], I32),
         "bitnet_linear_ex": ([P, I32, I64, I64, P, I64, P, P, F, P, I32, P, SZ, I32, P], I32),
@@ -312,6 +318,43 @@ def bitnet_linear_b1(x: torch.Tensor, Wp: torch.Tensor, beta: torch.Tensor, N: i
     return y
 
 
+def bitnet_t3_row_bytes(K: int) -> int:
+    return int(lib().bitnet_t3_row_bytes(K))
+
+
+def bitnet_pack_t3(Wq: torch.Tensor, n_invalid: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Base-3: five ternary weights per byte, [N, bitnet_t3_row_bytes(K)] uint8."""
+    N, K = Wq.shape
+    Wp = torch.empty((N, bitnet_t3_row_bytes(K)), dtype=torch.uint8, device=Wq.device)
+    _check(lib().bitnet_pack_t3(_ptr(Wq), N, K, _ptr(Wp), _ptr(n_invalid), _stream(stream)), "bitnet_pack_t3")
+    return Wp
+
+
+def bitnet_unpack_t3(Wp: torch.Tensor, K: int, n_invalid: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    N = Wp.shape[0]
+    Wq = torch.empty((N, K), dtype=torch.int8, device=Wp.device)
+    _check(lib().bitnet_unpack_t3(_ptr(Wp), N, K, _ptr(Wq), _ptr(n_invalid), _stream(stream)), "bitnet_unpack_t3")
+    return Wq
+
+
+def bitnet_linear_t3(x: torch.Tensor, Wp: torch.Tensor, gamma: torch.Tensor, N: int | None = None,
+                     rms_gain: torch.Tensor | None = None, rms_eps: float = 1e-5, y=None,
+                     y_dtype=torch.bfloat16, ws=None, stream=None):
+    """One token through base-3 packed weights."""
+    M, K = x.shape
+    if M != 1:
+        raise ValueError("bitnet_linear_t3 takes one token")
+    N = Wp.shape[0] if N is None else N
+    if y is None:
+        y = torch.empty((1, N), dtype=y_dtype, device=x.device)
+    if ws is None:
+        ws = new_workspace(bitnet_workspace_bytes(1, K, N), x.device)
+    _check(lib().bitnet_linear_t3(_ptr(x), _xdtype(x), K, _ptr(Wp), N, _ptr(gamma), _ptr(rms_gain),
+                                  float(rms_eps), _ptr(y), _ydtype(y.dtype), _ptr(ws), ws.numel(),
+                                  _stream(stream)), "bitnet_linear_t3")
+    return y
+
+
 def bitnet_quant_act_relu2(gate: torch.Tensor, up: torch.Tensor, rms_gain: torch.Tensor | None = None,
                            rms_eps: float = 1e-5, xq=None, x_scale=None, x_sum=None, stream=None):
     """Codes, scales and code sums of t = max(gate, 0)^2 * up."""
@@ -402,11 +445,16 @@ class GroupedCall:
                                       None if gain is None else _ptr(gain).value, _ptr(y).value,
                                       x.shape[1], Wp.shape[0])
         self.n = len(problems)
-        self.bits = int(bits)   # 2: ternary codes (bitnet_pack); 1: BitNet b1 signs (bitnet_pack_b1)
+        self.bits = int(bits)   # 2: ternary codes (bitnet_pack); 1: BitNet b1 signs (bitnet_pack_b1); 3: base-3
         self.eps = float(rms_eps)
         self.ws = ws if ws is not None else new_workspace(256, problems[0][0].device)
 
     def __call__(self, stream=None):
+        if self.bits == 3:
+            _check(lib().bitnet_linear_grouped_t3(ctypes.cast(self.arr, ctypes.c_void_p), self.n, self.xd, self.eps,
+                                                  self.yd, _ptr(self.ws), self.ws.numel(), _stream(stream)),
+                   "bitnet_linear_grouped_t3")
+            return
         if self.bits == 1:
             _check(lib().bitnet_linear_grouped_b1(ctypes.cast(self.arr, ctypes.c_void_p), self.n, self.xd, self.eps,
                                                   self.yd, _ptr(self.ws), self.ws.numel(), _stream(stream)),

@@ -276,10 +276,11 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
   const int64_t esz = prequant ? 1 : (x_dtype == BITNET_BF16 ? 2 : 4);
   p.bits = bits;
   for (int i = 0; i < count; ++i) {
-    if (pr[i].K % (64 * (3 - bits)) != 0) return BITNET_ERR_UNSUPPORTED;   // 16-byte packed rows
-    total += pr[i].N * (pr[i].K / 8 * bits);
-    max_rowb = std::max<int64_t>(max_rowb, pr[i].K / 8 * bits);
-    Kmax = std::max<int64_t>(Kmax, pr[i].K);
+    // 16-byte packed rows: K % 64 (2-bit), K % 128 (1-bit); base-3 rows are padded
+    if ((bits == 2 && pr[i].K % 64 != 0) || (bits == 1 && pr[i].K % 128 != 0)) return BITNET_ERR_UNSUPPORTED;
+    total += pr[i].N * gs_row_bytes(pr[i].K, bits);
+    max_rowb = std::max<int64_t>(max_rowb, gs_row_bytes(pr[i].K, bits));
+    Kmax = std::max<int64_t>(Kmax, gs_code_row(static_cast<int>(pr[i].K), bits));
     xmax = std::max<int64_t>(xmax, M * pr[i].K * esz);
   }
   p.total_bytes = total;
@@ -294,8 +295,9 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
   p.Kp_max = static_cast<int>(Kmax);
   // single-token activations are stored block-permuted for the lane-group
   // tasks; pre-quantised codes are copied as they are (warp tasks)
-  p.blocked = (pl.MT == 1 && !prequant) ? (bits == 2 ? 1 : 2) : 0;
-  if (bits == 1 && p.blocked != 2) return BITNET_ERR_UNSUPPORTED;   // 1-bit GEMV: one token, raw x
+  p.blocked = (pl.MT == 1 && !prequant && bits != 3) ? (bits == 2 ? 1 : 2) : 0;
+  // 1-bit and base-3 GEMV: one token, raw activations
+  if (bits != 2 && (pl.MT != 1 || prequant)) return BITNET_ERR_UNSUPPORTED;
   (void)xmax;
   // Shapes, most preferred first: (activation buffers, slots per warp, budget).
   // Two activation buffers let the activation warp run a segment ahead.
@@ -337,13 +339,16 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
     g.resid = pr[i].resid;
     g.K = static_cast<int>(pr[i].K);
     g.N = static_cast<int>(pr[i].N);
-    const int64_t rowb = pr[i].K / 8 * bits;
+    const int64_t rowb = gs_row_bytes(pr[i].K, bits);
     int64_t rc = slot / rowb;
     // a short stream: about one chunk per consumer warp
     if (!big) rc = std::min<int64_t>(rc, ((per_cta + rowb - 1) / rowb + kGsCW - 1) / kGsCW);
     rc = std::max<int64_t>(1, std::min<int64_t>(rc, pr[i].N));
     int task;
-    if (p.blocked) {
+    if (bits == 3) {
+      task = kGsTaskT3;
+      if (rc >= 4) rc -= rc % 4;
+    } else if (p.blocked) {
       // the largest lane-group task whose rows fit the chunk
       task = rc >= 8 ? kGsTaskG8R2 : (rc >= 4 ? kGsTaskG16R2 : (rc >= 2 ? kGsTaskG16R1 : kGsTaskG32R1));
       const int64_t unit = task == kGsTaskG8R2 ? 8 : (task == kGsTaskG16R2 ? 4 : (task == kGsTaskG16R1 ? 2 : 1));
@@ -712,10 +717,15 @@ static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in
     if (K % 128 != 0) return BITNET_ERR_SHAPE;
     gemv_ok = (M == 1 && x != nullptr);
   }
+  // base-3: one token through the streaming GEMV only (a decode format)
+  if (bits == 3) {
+    if (M != 1 || x == nullptr) return BITNET_ERR_UNSUPPORTED;
+    gemv_ok = true;
+  }
   if (path == BITNET_PATH_GEMV && !gemv_ok) return BITNET_ERR_UNSUPPORTED;
   const bool use_gemv = (path == BITNET_PATH_GEMV) || (path == BITNET_PATH_AUTO && gemv_ok);
 
-  if (use_gemv && K % 64 == 0) {
+  if (use_gemv && (K % 64 == 0 || bits == 3)) {
     StreamProblem sp{x != nullptr ? x : static_cast<const void*>(xq_in), Wp, gamma, rms_gain, scale_in, y, acc, K, N,
                      x2, resid};
     auto* pl = new (std::nothrow) StreamPlan<kStreamSmallP>;
@@ -847,7 +857,7 @@ static bitnet_status grouped_impl(const bitnet_gemv_problem* problems, int count
   if (count < 1 || count > kStreamMaxP) return BITNET_ERR_SHAPE;
   if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
   if (y_dtype != BITNET_F32 && y_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
-  if (M < 1 || M > (bits == 1 ? 1 : kGemvMaxM)) return BITNET_ERR_SHAPE;
+  if (M < 1 || M > (bits != 2 ? 1 : kGemvMaxM)) return BITNET_ERR_SHAPE;
   if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0 || ws_bytes < kWsHeader) return BITNET_ERR_WORKSPACE;
   std::vector<StreamProblem> sp(count);
   for (int i = 0; i < count; ++i) {
@@ -855,7 +865,7 @@ static bitnet_status grouped_impl(const bitnet_gemv_problem* problems, int count
     if (q.x == nullptr || q.Wp == nullptr || q.gamma == nullptr || q.y == nullptr) return BITNET_ERR_NULL;
     bitnet_status s = check_shape(M, q.K, q.N);
     if (s != BITNET_OK) return s;
-    if (q.K % (64 * (3 - bits)) != 0) return BITNET_ERR_SHAPE;
+    if ((bits == 2 && q.K % 64 != 0) || (bits == 1 && q.K % 128 != 0)) return BITNET_ERR_SHAPE;
     if (!aligned16(q.x) || !aligned16(q.Wp) || !aligned16(q.y) || (q.rms_gain != nullptr && !aligned16(q.rms_gain)))
       return BITNET_ERR_ALIGN;
     sp[i] = StreamProblem{q.x, q.Wp, q.gamma, q.rms_gain, nullptr, q.y, nullptr, q.K, q.N};
@@ -899,6 +909,52 @@ bitnet_status bitnet_linear_grouped(const bitnet_gemv_problem* problems, int cou
 bitnet_status bitnet_linear_grouped_b1(const bitnet_gemv_problem* problems, int count, int x_dtype, float rms_eps,
                                        int y_dtype, void* ws, size_t ws_bytes, bitnet_stream_t stream) {
   return grouped_impl(problems, count, 1, x_dtype, rms_eps, y_dtype, ws, ws_bytes, stream, 1);
+}
+
+bitnet_status bitnet_linear_grouped_t3(const bitnet_gemv_problem* problems, int count, int x_dtype, float rms_eps,
+                                       int y_dtype, void* ws, size_t ws_bytes, bitnet_stream_t stream) {
+  return grouped_impl(problems, count, 1, x_dtype, rms_eps, y_dtype, ws, ws_bytes, stream, 3);
+}
+
+int64_t bitnet_t3_row_bytes(int64_t K) { return K < 1 ? 0 : gs_row_bytes(K, 3); }
+
+bitnet_status bitnet_pack_t3(const int8_t* Wq, int64_t N, int64_t K, uint8_t* Wp, uint32_t* n_invalid,
+                             bitnet_stream_t stream) {
+  if (Wq == nullptr || Wp == nullptr) return BITNET_ERR_NULL;
+  if (check_shape(1, K, N) != BITNET_OK) return BITNET_ERR_SHAPE;
+  if (!aligned16(Wp)) return BITNET_ERR_ALIGN;
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  const int64_t rb = gs_row_bytes(K, 3);
+  pack_t3_kernel<<<elementwise_grid(N * rb / 4, d), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      Wq, N, K, rb, reinterpret_cast<uint32_t*>(Wp), n_invalid);
+  return launch_result(cudaSuccess);
+}
+
+bitnet_status bitnet_unpack_t3(const uint8_t* Wp, int64_t N, int64_t K, int8_t* Wq, uint32_t* n_invalid,
+                               bitnet_stream_t stream) {
+  if (Wq == nullptr || Wp == nullptr) return BITNET_ERR_NULL;
+  if (check_shape(1, K, N) != BITNET_OK) return BITNET_ERR_SHAPE;
+  if (!aligned16(Wp)) return BITNET_ERR_ALIGN;
+  DeviceInfo* d;
+  bitnet_status s = device_info(&d);
+  if (s != BITNET_OK) return s;
+  const int64_t rb = gs_row_bytes(K, 3);
+  unpack_t3_kernel<<<elementwise_grid(N * rb / 4, d), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      reinterpret_cast<const uint32_t*>(Wp), N, K, rb, Wq, n_invalid);
+  return launch_result(cudaSuccess);
+}
+
+bitnet_status bitnet_linear_t3(const void* x, int x_dtype, int64_t K, const uint8_t* Wp, int64_t N,
+                               const float* gamma, const float* rms_gain, float rms_eps, void* y, int y_dtype,
+                               void* ws, size_t ws_bytes, bitnet_stream_t stream) {
+  if (x == nullptr || y == nullptr) return BITNET_ERR_NULL;
+  if (x_dtype != BITNET_F32 && x_dtype != BITNET_BF16) return BITNET_ERR_DTYPE;
+  if (!aligned16(x)) return BITNET_ERR_ALIGN;
+  return linear_impl(x, x_dtype, nullptr, nullptr, nullptr, 1, K, Wp, N, gamma, rms_gain, rms_eps, y, y_dtype,
+                     nullptr, ws, ws_bytes, BITNET_PATH_AUTO, reinterpret_cast<cudaStream_t>(stream), nullptr,
+                     nullptr, 3);
 }
 
 bitnet_status bitnet_watchdog_selftest(void* ws, size_t ws_bytes, uint32_t limit_us, bitnet_stream_t stream) {

@@ -52,6 +52,7 @@ constexpr int kGsTaskG16R1 = 2;     // 2-row tasks
 constexpr int kGsTaskG32R1 = 3;     // 1-row tasks
 constexpr int kGsTaskWarp = 4;      // whole warp over R = 4 / 2 / 1 rows (M = 1 / 2 / 4), linear codes
 constexpr int kGsTaskB1 = 5;        // 1-bit signs: kGsTaskB1 + (a G/RS shape above, 0 .. 3)
+constexpr int kGsTaskT3 = 9;        // base-3: whole warp over 4 rows, linear codes
 
 struct GsProblem {
   const void* x;          // [M, K] raw activations (x_dtype) or int8 codes (prequant)
@@ -79,7 +80,7 @@ struct GsParams {
   int slot_bytes, nslots;        // ring of each consumer warp
   int nxb;                       // activation code buffers (2: quantise a segment ahead)
   int blocked;                   // 1 / 2: codes block-permuted in 4 / 8 quarters (lane-group tasks)
-  int bits;                      // 2: ternary codes, 2 bits per weight; 1: BitNet b1 signs
+  int bits;                      // 2: ternary codes, 2 bits per weight; 1: BitNet b1 signs; 3: base-3
   int Kp_max;                    // int8 code rows in shared memory (K rounded up to 64)
   uint64_t limit_ns;
   uint32_t* status;
@@ -96,6 +97,17 @@ struct GsHeader {
   int abort;
 };
 
+// Bytes of one packed row and the code-row length in shared memory, by
+// weight format: bits 2 (ternary codes, K/4 bytes), 1 (BitNet b1 signs,
+// K/8 bytes) or 3 (base-3, five weights per byte, ceil(K/80) 16-byte chunks;
+// the code row is zero-padded to a multiple of 80).
+__host__ __device__ __forceinline__ int64_t gs_row_bytes(int64_t K, int bits) {
+  return bits == 3 ? (K + 79) / 80 * 16 : K / 8 * bits;
+}
+__host__ __device__ __forceinline__ int gs_code_row(int K, int bits) {
+  return bits == 3 ? (K + 79) / 80 * 80 : (K + 63) & ~63;
+}
+
 // First global row (problem, row) of CTA b's share of the weight bytes: the
 // first row that starts at or after byte total * b / gridDim.x (binary
 // search over the problems' byte ranges).
@@ -105,7 +117,7 @@ __device__ __forceinline__ void gs_cta_start(const GsParams<MAXP>& p, int b, int
   int lo = 0, hi = p.nprob;   // first problem whose bytes end after target
   while (lo < hi) {
     const int mid = (lo + hi) >> 1;
-    const int64_t end = p.prob[mid].byte0 + static_cast<int64_t>(p.prob[mid].K / 8 * p.bits) * p.prob[mid].N;
+    const int64_t end = p.prob[mid].byte0 + gs_row_bytes(p.prob[mid].K, p.bits) * p.prob[mid].N;
     if (target < end)
       hi = mid;
     else
@@ -114,7 +126,7 @@ __device__ __forceinline__ void gs_cta_start(const GsParams<MAXP>& p, int b, int
   prob = lo;
   row = 0;
   if (lo == p.nprob) return;
-  const int64_t rb = p.prob[lo].K / 8 * p.bits;
+  const int64_t rb = gs_row_bytes(p.prob[lo].K, p.bits);
   // target may sit inside the previous problem's last row (before byte0)
   const int64_t off = target > p.prob[lo].byte0 ? target - p.prob[lo].byte0 : 0;
   const int64_t r = (off + rb - 1) / rb;
@@ -302,6 +314,58 @@ __device__ __forceinline__ void gs_task_lg_b1(const uint8_t* wbase, int rc, int 
   }
 }
 
+// Base-3 weights, M = 1: a warp owns R rows; lane l takes the 20-weight
+// groups l, l + 32, ... of each.  Group g is one uint32 whose byte j holds
+// the codes of weights 20g + 4i + j as base-3 digits i = 0..4.  The digits
+// come out two bytes at a time in 16-bit lanes: floor(v / 3) = (v * 171) >> 9
+// for every byte value v, and v - 3 floor(v / 3) is the digit, so digit i of
+// the four bytes lines up four codes with the activation word at 20g + 4i
+// for dp4a.  The code row is zero-padded past K (padding weights code 1).
+// Rows [row0, row0 + R) of the chunk.
+template <int R>
+__device__ __forceinline__ void gs_task_t3(const uint8_t* wbase, int rc, int row0, int rowb, const int8_t* xs,
+                                           int lane, int xsum0, float gs0, const GsProblem& P, int r, int y_dtype) {
+  const int nr = min(R, rc - row0);
+  const int nword = rowb / 4;
+  const uint32_t* wb = reinterpret_cast<const uint32_t*>(wbase + static_cast<int64_t>(row0) * rowb);
+  const uint32_t* x32 = reinterpret_cast<const uint32_t*>(xs);
+  int a[R];
+#pragma unroll
+  for (int i = 0; i < R; ++i) a[i] = 0;
+  for (int g = lane; g < nword; g += 32) {
+    uint32_t xw[5];
+#pragma unroll
+    for (int d = 0; d < 5; ++d) xw[d] = x32[5 * g + d];
+#pragma unroll
+    for (int i = 0; i < R; ++i) {
+      const uint32_t w = (i < nr) ? wb[i * nword + g] : 0u;
+      uint32_t lo = w & 0x00FF00FFu, hi = (w >> 8) & 0x00FF00FFu;
+#pragma unroll
+      for (int d = 0; d < 5; ++d) {
+        const uint32_t ql = ((lo * 171u) >> 9) & 0x007F007Fu, qh = ((hi * 171u) >> 9) & 0x007F007Fu;
+        a[i] = dp4a_us((lo - 3u * ql) | ((hi - 3u * qh) << 8), xw[d], a[i]);
+        lo = ql;
+        hi = qh;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < R; ++i) a[i] = warp_sum(a[i]);
+#pragma unroll
+  for (int i = 0; i < R; ++i) {
+    if (lane == i && i < nr) {
+      const int64_t n = r + row0 + i;
+      const int accv = a[i] - xsum0;
+      if (P.acc != nullptr) P.acc[n] = accv;
+      if (P.y != nullptr) {
+        float o = __fmul_rn(__int2float_rn(accv), gs0);
+        if (P.resid != nullptr) o = __fadd_rn(load_y(P.resid, y_dtype, n), o);
+        store_y(P.y, y_dtype, n, o);
+      }
+    }
+  }
+}
+
 // Long rows or M > 1: a warp owns R rows, lane l walks code words l, l + 32, ...
 // Rows [row0, row0 + R) of the stage.
 template <int R, int MT>
@@ -442,7 +506,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
   uint8_t* myslots = wslots + static_cast<size_t>(warp) * p.nslots * p.slot_bytes;
   auto issue = [&](int slot) {
     const GsProblem& Q = p.prob[icur.q];
-    const int64_t rowb = Q.K / 8 * p.bits;
+    const int64_t rowb = gs_row_bytes(Q.K, p.bits);
     const uint32_t bytes = static_cast<uint32_t>(min(Q.rc, icur.r1 - icur.r) * rowb);
     mbar_expect_tx(&H.wfull[warp][slot], bytes);
     bulk_g2s(myslots + slot * p.slot_bytes, Q.Wp + static_cast<int64_t>(icur.r) * rowb, bytes, &H.wfull[warp][slot]);
@@ -501,13 +565,16 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
     const GsProblem& P = p.prob[cv == 0 ? pb : q1];
     int8_t* xs = xsbuf + cv * xs_stride;
     float sc[MT];
-    const int Kp = (P.K + 63) & ~63;
+    const int Kp = gs_code_row(P.K, p.bits);
     if (p.prequant) {
       ok = copy_codes(P, xs, Kp, sc, &H.q.qpart[0][0], kAll, 0, tid == CW * 32) && ok;
     } else {
       quant_rows<kAll, MT, 1, false, kGsBarAll, false>(static_cast<const char*>(P.x), p.x_dtype, P.K * esz, p.M,
                                                       P.K, P.gain, p.rms_eps, xs, Kp, H.q, sc, 0, p.blocked,
                                                       static_cast<const char*>(P.x2));
+    }
+    if (p.bits == 3) {   // zero the code row's padding past K (no thread above wrote there)
+      for (int k = P.K + tid; k < Kp; k += kAll) xs[k] = 0;
     }
     group_sync<kGsBarAll, kAll>();
     // the activation warp publishes the version; it reads the shared partials
@@ -543,7 +610,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
         break;
       }
       const GsProblem& P = p.prob[q];
-      const int Kp = (P.K + 63) & ~63;
+      const int Kp = gs_code_row(P.K, p.bits);
       int8_t* xs = xsbuf + b * xs_stride;
       float sc[MT];
       if (p.prequant) {
@@ -556,6 +623,8 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
                                                      P.K, P.gain, p.rms_eps, xs, Kp, H.qx, sc, CW * 32,
                                                      p.blocked, static_cast<const char*>(P.x2));
       }
+      if (p.bits == 3)
+        for (int k = P.K + lane; k < Kp; k += 32) xs[k] = 0;
       __syncwarp();
       if (lane == 0) {
 #pragma unroll
@@ -599,12 +668,12 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
     }
     const GsProblem& P = p.prob[q];
     const int8_t* xs = xsbuf + (v % p.nxb) * xs_stride;
-    const int Kp = (P.K + 63) & ~63;
+    const int Kp = gs_code_row(P.K, p.bits);
     const float gamma = (q == pb) ? __ldg(P.gamma) : gamma_next;
     if (q < qlast) gamma_next = __ldg(p.prob[q + 1].gamma);   // in flight during this segment
     const float gs0 = __fmul_rn(gamma, sc[0]);
     const int nword = P.K / 16;      // 32-bit code words (16 weights) per row
-    const int rowb = P.K / 8 * p.bits, nchunk = P.K / (64 * (3 - p.bits));   // 16-byte chunks per row
+    const int rowb = static_cast<int>(gs_row_bytes(P.K, p.bits)), nchunk = rowb / 16;   // 16-byte chunks per row
     while (cur.q == q) {
       if (!gs_wait(&H.wfull[warp][slot], phase, p.limit_ns, abort_flag)) {
         ok = false;
@@ -625,6 +694,9 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
       } else if (MT == 1 && P.task == kGsTaskG32R1) {
         for (int row0 = 0; row0 < rows; ++row0)
           gs_task_lg<32, 1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+      } else if (MT == 1 && P.task == kGsTaskT3) {
+        for (int row0 = 0; row0 < rows; row0 += 4)
+          gs_task_t3<4>(wb8, rows, row0, rowb, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
       } else if (MT == 1 && P.task >= kGsTaskB1) {
         if (P.task == kGsTaskB1 + kGsTaskG8R2) {
           for (int row0 = 0; row0 < rows; row0 += 8)

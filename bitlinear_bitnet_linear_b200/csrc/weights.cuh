@@ -304,6 +304,74 @@ __global__ void __launch_bounds__(256) unpack_b1_kernel(const uint32_t* __restri
   }
 }
 
+// Base-3 pack: five ternary weights per byte (3^5 = 243 <= 256).  Row n
+// takes row_bytes = ceil(K/80)*16 bytes; byte j of the uint32 group g holds
+// sum_i c(20g + 4i + j) 3^i, i = 0..4, with codes c = q + 1 (weights past K:
+// code 1).  Values outside {-1, 0, 1} are stored as code 1 and counted.
+// One thread per group.
+__global__ void __launch_bounds__(256) pack_t3_kernel(const int8_t* __restrict__ Wq, int64_t N, int64_t K,
+                                                      int64_t row_bytes, uint32_t* __restrict__ Wp,
+                                                      uint32_t* n_invalid) {
+  uint32_t bad = 0;
+  const int64_t gpr = row_bytes / 4, total = N * gpr;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = t / gpr, g = t - n * gpr;
+    const int8_t* row = Wq + n * K;
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t v = 0, p3 = 1;
+#pragma unroll
+      for (int i = 0; i < 5; ++i) {
+        const int64_t k = 20 * g + 4 * i + j;
+        uint32_t c = 1;
+        if (k < K) {
+          const int q = row[k];
+          if (q >= -1 && q <= 1)
+            c = static_cast<uint32_t>(q + 1);
+          else
+            ++bad;
+        }
+        v += c * p3;
+        p3 *= 3u;
+      }
+      word |= v << (8 * j);
+    }
+    Wp[t] = word;
+  }
+  if (n_invalid != nullptr && bad) atomicAdd(n_invalid, bad);
+}
+
+// Inverse of pack_t3_kernel for k < K; a byte above 242 is invalid: its
+// weights read as 0 and it is counted.
+__global__ void __launch_bounds__(256) unpack_t3_kernel(const uint32_t* __restrict__ Wp, int64_t N, int64_t K,
+                                                        int64_t row_bytes, int8_t* __restrict__ Wq,
+                                                        uint32_t* n_invalid) {
+  uint32_t bad = 0;
+  const int64_t gpr = row_bytes / 4, total = N * gpr;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = t / gpr, g = t - n * gpr;
+    const uint32_t word = __ldg(Wp + t);
+    int8_t* row = Wq + n * K;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t v = (word >> (8 * j)) & 0xffu;
+      const bool valid = v <= 242u;
+      if (!valid && 20 * g + j < K) ++bad;
+#pragma unroll
+      for (int i = 0; i < 5; ++i) {
+        const int64_t k = 20 * g + 4 * i + j;
+        const uint32_t c = v % 3u;
+        v /= 3u;
+        if (k < K) row[k] = valid ? static_cast<int8_t>(static_cast<int>(c) - 1) : static_cast<int8_t>(0);
+      }
+    }
+  }
+  if (n_invalid != nullptr && bad) atomicAdd(n_invalid, bad);
+}
+
 __global__ void stream_fence_kernel() {}
 
 }  // namespace bitnet

@@ -181,6 +181,40 @@ bitnet_status bitnet_linear_b1(const void *x, int x_dtype, int64_t M, int64_t K,
                                bitnet_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * Base-3 packing: five ternary weights per byte (3^5 = 243 <= 256), about
+ * 1.6 bits per weight ("Key Technologies ... BitNET Family", Memory
+ * Efficiency: 0.4 GB for the 2B model; Hacker News thread on "2 bits
+ * instead of 1.58").  A decode format: one token per call.  K % 16 == 0, as
+ * everywhere in this library (K need not be a multiple of 20 or 80).
+ * Layout (this library's): a row takes bitnet_t3_row_bytes(K) =
+ * ceil(K/80) * 16 bytes; byte j of the little-endian uint32 group g holds
+ * sum_i c(20g + 4i + j) 3^i (i = 0..4) with codes c = q + 1; weights past K
+ * code as 1 (q = 0).
+ * ------------------------------------------------------------------------ */
+int64_t bitnet_t3_row_bytes(int64_t K);
+
+/* Pack Wq [N, K] int8 in {-1, 0, 1} into Wp [N, bitnet_t3_row_bytes(K)].
+ * Values outside {-1, 0, 1} are stored as code 1 and counted into
+ * *n_invalid (device uint32, may be NULL, accumulated). */
+bitnet_status bitnet_pack_t3(const int8_t *Wq, int64_t N, int64_t K, uint8_t *Wp,
+                             uint32_t *n_invalid, bitnet_stream_t stream);
+
+/* Inverse of bitnet_pack_t3; a byte above 242 is invalid: its five weights
+ * read as 0 and it is counted into *n_invalid (may be NULL). */
+bitnet_status bitnet_unpack_t3(const uint8_t *Wp, int64_t N, int64_t K, int8_t *Wq,
+                               uint32_t *n_invalid, bitnet_stream_t stream);
+
+/* BitLinear forward of ONE token (x [1, K]) with base-3 packed weights:
+ * y[n] exactly as bitnet_linear would give with the same ternary weights.
+ * The streaming GEMV decodes the base-3 digits in registers.  ws:
+ * bitnet_workspace_bytes(1, K, N) bytes. */
+bitnet_status bitnet_linear_t3(const void *x, int x_dtype, int64_t K,
+                               const uint8_t *Wp, int64_t N, const float *gamma,
+                               const float *rms_gain, float rms_eps,
+                               void *y, int y_dtype, void *ws, size_t ws_bytes,
+                               bitnet_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * Per-call path.
  * ------------------------------------------------------------------------ */
 
@@ -318,6 +352,12 @@ bitnet_status bitnet_quant_weights_noalloc(const float *W, int64_t N, int64_t K,
  * gamma = beta), one token (M = 1), K % 128 == 0: each problem is computed
  * exactly as bitnet_linear_b1. */
 bitnet_status bitnet_linear_grouped_b1(const bitnet_gemv_problem *problems, int count, int x_dtype,
+                                       float rms_eps, int y_dtype, void *ws, size_t ws_bytes,
+                                       bitnet_stream_t stream);
+
+/* bitnet_linear_grouped for base-3 packed weights (bitnet_pack_t3), one
+ * token (M = 1): each problem is computed exactly as bitnet_linear_t3. */
+bitnet_status bitnet_linear_grouped_t3(const bitnet_gemv_problem *problems, int count, int x_dtype,
                                        float rms_eps, int y_dtype, void *ws, size_t ws_bytes,
                                        bitnet_stream_t stream);
 

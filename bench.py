@@ -38,9 +38,9 @@ sys.path.insert(0, ROOT)
 METRIC = "BitLinear decode GEMV HBM GB/s (% of peak); prefill GEMM int8 TOPS (% peak)"
 # DRAM bytes (read + write) per launch from one ncu capture of each kernel as
 # it stands (profiles/); set to None whenever the kernel changes.
-# Decode: 79.59 + 1.70 MB on the 4-layer stack, scaled by weight bytes to 30 layers.
-TRAFFIC_DECODE = round((79.593984e6 + 1.696256e6) * 597673800 / 79689840)
-TRAFFIC_PREFILL = None   # kernel changed since its capture
+# Decode: 79.61 + 1.79 MB on the 4-layer stack, scaled by weight bytes to 30 layers.
+TRAFFIC_DECODE = round((79.606272e6 + 1.786624e6) * 597673800 / 79689840)
+TRAFFIC_PREFILL = round(15.0336e6 + 5.80992e6)
 WORKLOAD = ("decode GEMV M=1 over the 2560x2560 / 2560x6912 / 6912x2560 BitLinear shapes, "
             "30-layer BitNet-b1.58-style stack (210 calls per token, 594.7 MB packed 2-bit weights)")
 NOMINAL_INT8_OVER_BF16 = 2.0        # dense int8 (as fp8) vs dense bf16, nominal B200 ratio

@@ -369,9 +369,9 @@ bitnet_status plan_stream(const DeviceInfo* d, const StreamProblem* pr, int coun
   return BITNET_OK;
 }
 
-template <int MT, int MAXP>
+template <int MT, int MAXP, int BITS>
 cudaError_t run_stream_t(const StreamPlan<MAXP>& pl, cudaStream_t st) {
-  auto k = gemv_stream_kernel<MT, MAXP, kGsCW>;
+  auto k = gemv_stream_kernel<MT, MAXP, kGsCW, BITS>;
   cudaError_t e = allow_smem(k, pl.smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(k, dim3(pl.grid), dim3(kGsCW * 32 + 32), pl.smem, st, pl.p);
@@ -379,10 +379,12 @@ cudaError_t run_stream_t(const StreamPlan<MAXP>& pl, cudaStream_t st) {
 
 template <int MAXP>
 cudaError_t run_stream(const StreamPlan<MAXP>& pl, cudaStream_t st) {
+  if (pl.p.bits == 1) return pl.MT == 1 ? run_stream_t<1, MAXP, 1>(pl, st) : cudaErrorInvalidValue;
+  if (pl.p.bits == 3) return pl.MT == 1 ? run_stream_t<1, MAXP, 3>(pl, st) : cudaErrorInvalidValue;
   switch (pl.MT) {
-    case 1: return run_stream_t<1, MAXP>(pl, st);
-    case 2: return run_stream_t<2, MAXP>(pl, st);
-    case 4: return run_stream_t<4, MAXP>(pl, st);
+    case 1: return run_stream_t<1, MAXP, 2>(pl, st);
+    case 2: return run_stream_t<2, MAXP, 2>(pl, st);
+    case 4: return run_stream_t<4, MAXP, 2>(pl, st);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -435,8 +435,13 @@ __device__ __forceinline__ void gs_task_warp(const uint32_t* wbase, int rc, int 
 }
 
 // CW consumer warps + one activation warp.
-template <int MT, int MAXP, int CW>
+// BITS (the weight format, 2 / 1 / 3 as GsParams::bits) is a template
+// parameter so that each instantiation holds only its own contraction
+// tasks: fewer code bytes in the consumers' loop, fewer instruction-cache
+// misses.
+template <int MT, int MAXP, int CW, int BITS>
 __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __grid_constant__ GsParams<MAXP> p) {
+  static_assert(BITS == 2 || MT == 1, "1-bit and base-3 weights: one token");
   constexpr int kAll = CW * 32 + 32;
   extern __shared__ __align__(128) uint8_t smem[];
   static_assert(sizeof(GsHeader<MT, CW>) <= kGsHeader, "header too large");
@@ -506,7 +511,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
   uint8_t* myslots = wslots + static_cast<size_t>(warp) * p.nslots * p.slot_bytes;
   auto issue = [&](int slot) {
     const GsProblem& Q = p.prob[icur.q];
-    const int64_t rowb = gs_row_bytes(Q.K, p.bits);
+    const int64_t rowb = gs_row_bytes(Q.K, BITS);
     const uint32_t bytes = static_cast<uint32_t>(min(Q.rc, icur.r1 - icur.r) * rowb);
     mbar_expect_tx(&H.wfull[warp][slot], bytes);
     bulk_g2s(myslots + slot * p.slot_bytes, Q.Wp + static_cast<int64_t>(icur.r) * rowb, bytes, &H.wfull[warp][slot]);
@@ -565,7 +570,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
     const GsProblem& P = p.prob[cv == 0 ? pb : q1];
     int8_t* xs = xsbuf + cv * xs_stride;
     float sc[MT];
-    const int Kp = gs_code_row(P.K, p.bits);
+    const int Kp = gs_code_row(P.K, BITS);
     if (p.prequant) {
       ok = copy_codes(P, xs, Kp, sc, &H.q.qpart[0][0], kAll, 0, tid == CW * 32) && ok;
     } else {
@@ -573,7 +578,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
                                                       P.K, P.gain, p.rms_eps, xs, Kp, H.q, sc, 0, p.blocked,
                                                       static_cast<const char*>(P.x2));
     }
-    if (p.bits == 3) {   // zero the code row's padding past K (no thread above wrote there)
+    if constexpr (BITS == 3) {   // zero the code row's padding past K (no thread above wrote there)
       for (int k = P.K + tid; k < Kp; k += kAll) xs[k] = 0;
     }
     group_sync<kGsBarAll, kAll>();
@@ -610,7 +615,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
         break;
       }
       const GsProblem& P = p.prob[q];
-      const int Kp = gs_code_row(P.K, p.bits);
+      const int Kp = gs_code_row(P.K, BITS);
       int8_t* xs = xsbuf + b * xs_stride;
       float sc[MT];
       if (p.prequant) {
@@ -623,7 +628,7 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
                                                      P.K, P.gain, p.rms_eps, xs, Kp, H.qx, sc, CW * 32,
                                                      p.blocked, static_cast<const char*>(P.x2));
       }
-      if (p.bits == 3)
+      if constexpr (BITS == 3)
         for (int k = P.K + lane; k < Kp; k += 32) xs[k] = 0;
       __syncwarp();
       if (lane == 0) {
@@ -668,12 +673,12 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
     }
     const GsProblem& P = p.prob[q];
     const int8_t* xs = xsbuf + (v % p.nxb) * xs_stride;
-    const int Kp = gs_code_row(P.K, p.bits);
+    const int Kp = gs_code_row(P.K, BITS);
     const float gamma = (q == pb) ? __ldg(P.gamma) : gamma_next;
     if (q < qlast) gamma_next = __ldg(p.prob[q + 1].gamma);   // in flight during this segment
     const float gs0 = __fmul_rn(gamma, sc[0]);
     const int nword = P.K / 16;      // 32-bit code words (16 weights) per row
-    const int rowb = static_cast<int>(gs_row_bytes(P.K, p.bits)), nchunk = rowb / 16;   // 16-byte chunks per row
+    const int rowb = static_cast<int>(gs_row_bytes(P.K, BITS)), nchunk = rowb / 16;   // 16-byte chunks per row
     while (cur.q == q) {
       if (!gs_wait(&H.wfull[warp][slot], phase, p.limit_ns, abort_flag)) {
         ok = false;
@@ -682,22 +687,10 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
       const uint8_t* wb8 = myslots + slot * p.slot_bytes;
       const int rows = min(P.rc, cur.r1 - cur.r);
       const int r = cur.r;
-      if (MT == 1 && P.task == kGsTaskG8R2) {
-        for (int row0 = 0; row0 < rows; row0 += 8)
-          gs_task_lg<8, 2>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
-      } else if (MT == 1 && P.task == kGsTaskG16R2) {
-        for (int row0 = 0; row0 < rows; row0 += 4)
-          gs_task_lg<16, 2>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
-      } else if (MT == 1 && P.task == kGsTaskG16R1) {
-        for (int row0 = 0; row0 < rows; row0 += 2)
-          gs_task_lg<16, 1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
-      } else if (MT == 1 && P.task == kGsTaskG32R1) {
-        for (int row0 = 0; row0 < rows; ++row0)
-          gs_task_lg<32, 1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
-      } else if (MT == 1 && P.task == kGsTaskT3) {
+      if constexpr (BITS == 3) {
         for (int row0 = 0; row0 < rows; row0 += 4)
           gs_task_t3<4>(wb8, rows, row0, rowb, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
-      } else if (MT == 1 && P.task >= kGsTaskB1) {
+      } else if constexpr (BITS == 1) {
         if (P.task == kGsTaskB1 + kGsTaskG8R2) {
           for (int row0 = 0; row0 < rows; row0 += 8)
             gs_task_lg_b1<8, 2>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
@@ -711,6 +704,18 @@ __global__ void __launch_bounds__(CW * 32 + 32, 1) gemv_stream_kernel(const __gr
           for (int row0 = 0; row0 < rows; ++row0)
             gs_task_lg_b1<32, 1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
         }
+      } else if (MT == 1 && P.task == kGsTaskG8R2) {
+        for (int row0 = 0; row0 < rows; row0 += 8)
+          gs_task_lg<8, 2>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+      } else if (MT == 1 && P.task == kGsTaskG16R2) {
+        for (int row0 = 0; row0 < rows; row0 += 4)
+          gs_task_lg<16, 2>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+      } else if (MT == 1 && P.task == kGsTaskG16R1) {
+        for (int row0 = 0; row0 < rows; row0 += 2)
+          gs_task_lg<16, 1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
+      } else if (MT == 1 && P.task == kGsTaskG32R1) {
+        for (int row0 = 0; row0 < rows; ++row0)
+          gs_task_lg<32, 1>(wb8, rows, row0, rowb, nchunk, xs, lane, xsum[0], gs0, P, r, p.y_dtype);
       } else {
         constexpr int R = (MT == 1) ? 4 : ((MT == 2) ? 2 : 1);
         const uint32_t* wbase = reinterpret_cast<const uint32_t*>(wb8);

@@ -38,8 +38,8 @@ sys.path.insert(0, ROOT)
 METRIC = "BitLinear decode GEMV HBM GB/s (% of peak); prefill GEMM int8 TOPS (% peak)"
 # DRAM bytes (read + write) per launch from one ncu capture of each kernel as
 # it stands (profiles/); set to None whenever the kernel changes.
-# Decode: 79.61 + 1.79 MB on the 4-layer stack, scaled by weight bytes to 30 layers.
-TRAFFIC_DECODE = round((79.606272e6 + 1.786624e6) * 597673800 / 79689840)
+# Decode: 79.60 + 3.28 MB on the 4-layer stack, scaled by weight bytes to 30 layers.
+TRAFFIC_DECODE = round((79.602688e6 + 3.279872e6) * 597673800 / 79689840)
 TRAFFIC_PREFILL = round(15.0336e6 + 5.80992e6)
 WORKLOAD = ("decode GEMV M=1 over the 2560x2560 / 2560x6912 / 6912x2560 BitLinear shapes, "
             "30-layer BitNet-b1.58-style stack (210 calls per token, 594.7 MB packed 2-bit weights)")
@@ -399,8 +399,11 @@ def run_ours(args):
         d2h = sum(y.numel() * 2 for y in ys)
         x_pin = torch.cat([x.reshape(-1) for x in xs_host]).pin_memory()
         y_pin = torch.empty(sum(y.numel() for y in ys), dtype=torch.bfloat16).pin_memory()
-        x_dev = torch.empty_like(x_pin, device=dev)
-        y_dev = torch.empty(y_pin.numel(), dtype=torch.bfloat16, device=dev)
+        # two device buffer sets, so step t's kernel overlaps the H2D copy of
+        # step t + 1 and the D2H copy of step t - 1 (copy streams, events);
+        # every step still moves its own inputs and result across the bus
+        x_dev = [torch.empty_like(x_pin, device=dev) for _ in range(2)]
+        y_dev = [torch.empty(y_pin.numel(), dtype=torch.bfloat16, device=dev) for _ in range(2)]
         xo, yo = [], []
         o = 0
         for x in xs_host:
@@ -410,35 +413,48 @@ def run_ours(args):
         for y in ys:
             yo.append((o, y.shape[1]))
             o += y.numel()
-        xviews = [x_dev[a:a + k].view(1, k) for a, k in xo]
-        yviews = [y_dev[a:a + n].view(1, n) for a, n in yo]
-        eproblems = [(x, Wp, g, gains[K], y) for (K, N, Wp, g), x, y in zip(stack, xviews, yviews)]
+        ecalls = []
+        for bsel in range(2):
+            xviews = [x_dev[bsel][a:a + k].view(1, k) for a, k in xo]
+            yviews = [y_dev[bsel][a:a + n].view(1, n) for a, n in yo]
+            eproblems = [(x, Wp, g, gains[K], y) for (K, N, Wp, g), x, y in zip(stack, xviews, yviews)]
+            ecalls.append(bn.GroupedCall(eproblems, rms_eps=1e-5, ws=ws))
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_k = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-        ecall = bn.GroupedCall(eproblems, rms_eps=1e-5, ws=ws)
-
-        def e2e_step():
-            x_dev.copy_(x_pin, non_blocking=True)
-            ecall()
-            y_pin.copy_(y_dev, non_blocking=True)
+        def e2e_run(n):
+            for i in range(n):
+                bsel = i & 1
+                s_in.wait_event(ev_k[bsel])                 # x buffer read by the kernel two steps back
+                with torch.cuda.stream(s_in):
+                    x_dev[bsel].copy_(x_pin, non_blocking=True)
+                ev_in[bsel].record(s_in)
+                stream.wait_event(ev_in[bsel])
+                stream.wait_event(ev_out[bsel])            # y buffer copied out two steps back
+                ecalls[bsel](stream)
+                ev_k[bsel].record(stream)
+                s_out.wait_event(ev_k[bsel])
+                with torch.cuda.stream(s_out):
+                    y_pin.copy_(y_dev[bsel], non_blocking=True)
+                ev_out[bsel].record(s_out)
 
         e2e_steps = max(10, min(500, args.steps // 4))
-        with torch.cuda.stream(stream):
-            for _ in range(3):
-                e2e_step()
+        e2e_run(4)
         barrier()
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for _ in range(e2e_steps):
-                e2e_step()
-            e1.record(stream)
+        e0.record(s_in)
+        e2e_run(e2e_steps)
+        e1.record(s_out)
         barrier()
         ems = replicas.max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dev)
         e2e = {"value": round(replicas.whole_job_rate(bytes_step, world, ems * 1e-3) / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(ems, 4),
-               "path": "python binding (prepared GroupedCall) -> C ABI bitnet_linear_grouped (210 problems), "
-                       "one pinned host copy of all x in, one of all y out, no graph"}
+               "path": "python binding (prepared GroupedCall) -> C ABI bitnet_linear_grouped (210 problems); "
+                       "per step one pinned-host copy of all x in and one of all y out, on copy streams that "
+                       "overlap the neighbouring steps' kernels (two device buffer sets), no graph"}
 
     # ---- prefill GEMM (secondary) ------------------------------------------
     prefill = None

@@ -72,7 +72,7 @@ def b1_weights(N, K, seed):
 # M = 1: the streaming GEMV (1-bit lane groups); M > 1: the tensor-core path
 @pytest.mark.parametrize("M,K,N", [(1, 2560, 2560), (1, 6912, 2560), (1, 2560, 6912), (1, 128, 37),
                                    (1, 8192, 640), (2, 2560, 384), (64, 2560, 1000), (300, 6912, 512),
-                                   (5, 384, 130)])
+                                   (5, 384, 130), (600, 2560, 300)])
 @pytest.mark.parametrize("with_gain", [False, True])
 def test_linear_b1_matches_oracle(M, K, N, with_gain):
     x = synthetic.activations(M, K, seed=500 + M + K, dtype=torch.bfloat16)

@@ -56,7 +56,7 @@ def test_quant_act_relu2_bitexact(M, K, dtype, with_gain):
 
 # M <= 4 with K % 64 == 0: the streaming GEMV; otherwise the tensor-core path
 @pytest.mark.parametrize("M,K,N", [(1, 6912, 2560), (2, 2560, 1000), (4, 6912, 256), (16, 2560, 384),
-                                   (300, 2560, 512), (3, 272, 130)])
+                                   (300, 2560, 512), (3, 272, 130), (520, 2560, 200)])
 @pytest.mark.parametrize("y_dtype", [torch.float32, torch.bfloat16])
 @pytest.mark.parametrize("with_resid", [False, True])
 def test_linear_relu2_matches_oracle(M, K, N, y_dtype, with_resid):

@@ -171,6 +171,8 @@ ACC_CASES = [
     (1, 256, 256), (1, 2560, 2560), (2, 2560, 6912), (3, 272, 257), (4, 6912, 2560), (4, 336, 1),
     (1, 16, 5), (5, 2560, 300), (16, 128, 128), (17, 272, 129), (64, 2560, 6912), (100, 336, 129),
     (129, 1024, 1000), (257, 2560, 384), (300, 64, 200),
+    # 512 tokens and more: tiles of 128 weight rows x 256 tokens, ragged in both
+    (512, 256, 128), (600, 1024, 1000), (777, 272, 129),
 ]
 
 
@@ -207,6 +209,8 @@ E2E_CASES = [
     (16, 2560, 6912, torch.bfloat16, torch.bfloat16, True),
     (64, 2560, 6912, torch.bfloat16, torch.bfloat16, True),
     (200, 336, 130, torch.float32, torch.bfloat16, False),
+    (700, 336, 130, torch.float32, torch.bfloat16, False),
+    (530, 2560, 1000, torch.bfloat16, torch.float32, True),
 ]
 
 

@@ -344,21 +344,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // converter arrivals), dfull[b] (all MMAs of a tile done), dfree[b] (8
 // epilogue warps done reading buffer b), mdone (every MMA issued has
 // completed, before TMEM is freed).
+//
+// TA = true keeps the expanded codes out of shared memory: the converters
+// write them to TMEM with tcgen05.st and the MMAs take A from there (the TS
+// form), so shared memory carries only the activation tiles.  TMEM then
+// holds three accumulator slots of BM columns and AS A stages of 64 columns
+// (two halves of 32).  Tile i accumulates its weight-row halves in slots
+// 2i mod 3 and (2i + 1) mod 3; tile i + 1 takes the third slot and tile i's
+// first, so its MMAs start as soon as the epilogue has read tile i's first
+// half (dfree[s]: slot s read by all 8 epilogue warps, which drain the two
+// halves in order, each warp 64 tokens of one TMEM lane quadrant).
 // ---------------------------------------------------------------------------
 constexpr int kTpRows = 256;
 constexpr int kTpThreads = 18 * 32;
 constexpr int kTpAStage = kTpRows * kTcBK;     // 32 KB of expanded codes per K block
 
-template <int BM, int SS, int AS>
+template <int BM, int SS, int AS, bool TA = false>
 __host__ __device__ constexpr int tp_smem_bytes() {
-  return 1024 /* alignment slack */ + SS * BM * kTcBK + AS * kTpAStage + 1024 /* barriers, flags */;
+  return 1024 /* alignment slack */ + SS * BM * kTcBK + (TA ? 0 : AS * kTpAStage) + 1024 /* barriers, flags */;
 }
 
-template <int BM, int SS, int AS, int BITS = 2>
+template <int BM, int SS, int AS, int BITS = 2, bool TA = false>
 __global__ void __launch_bounds__(kTpThreads, 1)
     tc_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
-  static_assert(BM == 128, "two buffers of 2 x BM accumulator columns fill TMEM");
+  static_assert(BM == 128 && (!TA || 3 * BM + 64 * AS <= 512),
+                "the accumulators (and the TMEM A stages) fit the 512 TMEM columns");
   constexpr uint32_t kCols = 512;
+  constexpr int kDB = TA ? 1 : 2;                      // tile-completion barriers in turn
+  constexpr uint32_t kACol0 = 3 * BM;                  // TA: A stage a at [3 BM + 64 a, 3 BM + 64 a + 64)
+  constexpr int kASmem = TA ? 0 : kTpAStage;           // shared-memory bytes of one A stage
   constexpr uint32_t kStageBytes = BM * kTcBK;
   constexpr uint32_t kIdesc = idesc_i8_us(kTcBN, BM);
   constexpr int kPD = 4;                               // converter prefetch depth (K blocks)
@@ -367,13 +381,13 @@ __global__ void __launch_bounds__(kTpThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = smem;
   uint8_t* as = smem + SS * kStageBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(as + AS * kTpAStage);
+  uint64_t* full = reinterpret_cast<uint64_t*>(as + AS * kASmem);
   uint64_t* sempty = full + SS;
   uint64_t* afull = sempty + SS;
   uint64_t* aempty = afull + AS;
   uint64_t* dfull = aempty + AS;
   uint64_t* dfree = dfull + 2;
-  uint64_t* mdone = dfree + 2;
+  uint64_t* mdone = dfree + 3;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mdone + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
@@ -397,10 +411,8 @@ __global__ void __launch_bounds__(kTpThreads, 1)
       mbar_init(&afull[a], 256);
       mbar_init(&aempty[a], 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&dfull[b], 1);
-      mbar_init(&dfree[b], 8);
-    }
+    for (int b = 0; b < 2; ++b) mbar_init(&dfull[b], 1);
+    for (int b = 0; b < 3; ++b) mbar_init(&dfree[b], 8);
     mbar_init(mdone, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -450,16 +462,33 @@ __global__ void __launch_bounds__(kTpThreads, 1)
     if (lane == 0) {
       bool ok = true;
       int g = 0;
+      uint32_t slot_par = 0;   // TA: bit s = parity of the uses of slot s so far
       for (int i = 0; i < my_tiles && ok; ++i) {
-        const int b = i & 1;
-        // the epilogue has read what the tile before last left in buffer b
-        if (!mbar_wait_sleep(&dfree[b], ((i >> 1) & 1) ^ 1u, p.limit_ns, abort_flag)) {
-          if (!*abort_flag) fail(0x312u);
-          ok = false;
-          break;
+        const int b = i % kDB;
+        uint32_t d0, d1;         // accumulators of the two weight-row halves
+        if constexpr (TA) {
+          const int s0 = (2 * i) % 3, s1 = (2 * i + 1) % 3;
+          // the epilogue has read what earlier tiles left in both slots
+          if (!mbar_wait_sleep(&dfree[s0], ((slot_par >> s0) & 1u) ^ 1u, p.limit_ns, abort_flag) ||
+              !mbar_wait_sleep(&dfree[s1], ((slot_par >> s1) & 1u) ^ 1u, p.limit_ns, abort_flag)) {
+            if (!*abort_flag) fail(0x312u);
+            ok = false;
+            break;
+          }
+          slot_par ^= (1u << s0) | (1u << s1);
+          d0 = tmem + static_cast<uint32_t>(s0 * BM);
+          d1 = tmem + static_cast<uint32_t>(s1 * BM);
+        } else {
+          // the epilogue has read what the tile before last left in buffer b
+          if (!mbar_wait_sleep(&dfree[b], ((i >> 1) & 1) ^ 1u, p.limit_ns, abort_flag)) {
+            if (!*abort_flag) fail(0x312u);
+            ok = false;
+            break;
+          }
+          d0 = tmem + static_cast<uint32_t>(b * 2 * BM);
+          d1 = d0 + BM;
         }
         tc_fence_after();
-        const uint32_t d0 = tmem + static_cast<uint32_t>(b * 2 * BM);
         for (int kb = 0; kb < KB; ++kb, ++g) {
           const int s = g % SS;
           const int a = g % AS;
@@ -472,14 +501,25 @@ __global__ void __launch_bounds__(kTpThreads, 1)
           }
           tc_fence_after();
           const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xs + s * kStageBytes));
-          const uint64_t adesc0 = smem_desc_k_sw128(smem_u32(as + a * kTpAStage));
-          const uint64_t adesc1 = smem_desc_k_sw128(smem_u32(as + a * kTpAStage + kTpAStage / 2));
+          if constexpr (TA) {
+            const uint32_t a0 = tmem + kACol0 + 64u * static_cast<uint32_t>(a);
 #pragma unroll
-          for (int j = 0; j < kTcBK / 32; ++j) {
-            // K step of 32 bytes: advance both descriptors' start address by 32 B (>> 4 = 2)
-            const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
-            tc_mma_i8_ss(d0, adesc0 + 2ull * j, bdesc + 2ull * j, kIdesc, acc);
-            tc_mma_i8_ss(d0 + BM, adesc1 + 2ull * j, bdesc + 2ull * j, kIdesc, acc);
+            for (int j = 0; j < kTcBK / 32; ++j) {
+              // K step of 32 bytes: 8 TMEM columns of A, 32 B of the B descriptor (>> 4 = 2)
+              const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
+              tc_mma_i8_ts(d0, a0 + 8u * j, bdesc + 2ull * j, kIdesc, acc);
+              tc_mma_i8_ts(d1, a0 + 32u + 8u * j, bdesc + 2ull * j, kIdesc, acc);
+            }
+          } else {
+            const uint64_t adesc0 = smem_desc_k_sw128(smem_u32(as + a * kTpAStage));
+            const uint64_t adesc1 = smem_desc_k_sw128(smem_u32(as + a * kTpAStage + kTpAStage / 2));
+#pragma unroll
+            for (int j = 0; j < kTcBK / 32; ++j) {
+              // K step of 32 bytes: advance both descriptors' start address by 32 B (>> 4 = 2)
+              const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
+              tc_mma_i8_ss(d0, adesc0 + 2ull * j, bdesc + 2ull * j, kIdesc, acc);
+              tc_mma_i8_ss(d1, adesc1 + 2ull * j, bdesc + 2ull * j, kIdesc, acc);
+            }
           }
           tc_commit(&sempty[s]);
           tc_commit(&aempty[a]);
@@ -493,7 +533,12 @@ __global__ void __launch_bounds__(kTpThreads, 1)
     pdl_launch_dependents();
   } else if (warp < 10) {
     // ------------------------------------------------------------ converters
-    const int row = (warp - 2) * 32 + lane;          // A row of the 256-row tile
+    // A row of the 256-row tile.  TA: warp w may only reach TMEM lanes
+    // [32 (w % 4), 32 (w % 4) + 32), so it takes rows of lane quadrant w % 4
+    // in half (w - 2) / 4.
+    const int row = TA ? ((warp - 2) >> 2) * 128 + (warp & 3) * 32 + lane : (warp - 2) * 32 + lane;
+    const uint32_t a_lane_col = (static_cast<uint32_t>((warp & 3) * 32) << 16) + kACol0 +
+                                32u * static_cast<uint32_t>((warp - 2) >> 2);
     const int rowbytes = p.K * BITS / 8;
     const int total = my_tiles * KB;
     uint32_t wb[kPD][8];
@@ -519,7 +564,29 @@ __global__ void __launch_bounds__(kTpThreads, 1)
           if (!mbar_wait_sleep(&aempty[a], ((g / AS) & 1) ^ 1u, p.limit_ns, abort_flag)) {
             if (!*abort_flag) fail(0x314u);
             ok = false;
-          } else {
+          }
+          if constexpr (TA) {
+            // tcgen05.st is warp-collective: the warp goes on only together
+            // (the waits return together unless aborting)
+            if (__all_sync(0xffffffffu, ok)) {
+              uint32_t codes[32];
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                const uint4 c4 = tc_expand_chunk<BITS>(wb[j], c);
+                codes[4 * c + 0] = c4.x;
+                codes[4 * c + 1] = c4.y;
+                codes[4 * c + 2] = c4.z;
+                codes[4 * c + 3] = c4.w;
+              }
+              tmem_st_32x32b_x32(tmem + a_lane_col + 64u * static_cast<uint32_t>(a), codes);
+              tc_wait_st();
+              tc_fence_before();
+              mbar_arrive(&afull[a]);
+              if (g + kPD < total) load(g + kPD, wb[j]);
+            } else {
+              ok = false;
+            }
+          } else if (ok) {
             uint8_t* arow = as + a * kTpAStage + row * kTcBK;
 #pragma unroll
             for (int c = 0; c < 8; ++c)   // chunk c: weights 16c .. 16c + 15 of the K block
@@ -536,11 +603,16 @@ __global__ void __launch_bounds__(kTpThreads, 1)
     pdl_launch_dependents();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int h = (warp - 10) >> 2;
+    // Shared-memory A: warp w drains all BM tokens of weight-row half
+    // (w - 10) / 4.  TMEM A: warp w drains tokens [64 t, 64 t + 64),
+    // t = (w - 10) / 4, of both halves, the first half's slot first.
+    // Either way the warp reads TMEM lane quadrant w % 4.
     const int q = warp & 3;
-    const int row = h * 128 + q * 32 + lane;
+    const int h_own = TA ? 0 : (warp - 10) >> 2;
+    const int tok0 = TA ? ((warp - 10) >> 2) * 64 : 0;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    constexpr int kChunks = BM / 32;
+    constexpr int kChunks = (TA ? 64 : BM) / 32;
+    constexpr int kHalves = TA ? 2 : 1;
     const bool fast = p.y != nullptr && p.acc == nullptr && p.resid == nullptr && p.y_dtype == BITNET_BF16 &&
                       p.K <= 32768;
     pdl_wait();   // token scales and sums come from the previous kernel
@@ -548,10 +620,11 @@ __global__ void __launch_bounds__(kTpThreads, 1)
     const float* __restrict__ xsc = p.x_scale;
     const int32_t* __restrict__ xsm = p.x_sum;
     for (int i = 0; i < my_tiles; ++i) {
-      const int b = i & 1;
-      const int m0 = tile_m0(i);
-      const int n = tile_n0(i) + row;
-      const bool valid = n < p.N;
+      const int b = i % kDB;
+      const int u = i / kDB;   // earlier uses of barrier b
+      const int m0 = tile_m0(i) + tok0;   // this warp's first token
+      // chunks of 32 tokens holding tokens below M (warp-uniform)
+      const int nc = min(kChunks, (max(0, p.M - m0) + 31) / 32);
       // lane l holds token (m0 + 32 c + l)'s scale and code sum: loaded before
       // the accumulators are ready, shuffled out below
       float gs[kChunks];
@@ -566,63 +639,84 @@ __global__ void __launch_bounds__(kTpThreads, 1)
           xsum[c] = __ldg(xsm + mi);
         }
       }
-      const bool got = mbar_wait_sleep(&dfull[b], (i >> 1) & 1, p.limit_ns, abort_flag);
+      const bool got = mbar_wait_sleep(&dfull[b], u & 1, p.limit_ns, abort_flag);
       if (!got && !*abort_flag) fail(0x315u);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       if (i + 1 == my_tiles) pdl_launch_dependents();
-      const uint32_t dcol = static_cast<uint32_t>(b * 2 * BM + h * BM);
-      // A rolled loop over the 32-token chunks keeps the (unrolled) chunk
-      // body in the instruction cache: fully unrolled, the epilogue is
-      // straight-line code that runs once per tile and misses on every fetch.
 #pragma unroll 1
-      for (int c = 0; c < kChunks; ++c) {
-        if (m0 + 32 * c >= p.M) break;   // warp-uniform
-        float gsc = gs[0];
-        int xsc_ = xsum[0];
+      for (int hh = 0; hh < kHalves; ++hh) {
+        const int h = TA ? hh : h_own;                 // weight-row half
+        const int slot = TA ? (2 * i + hh) % 3 : 0;    // TA: its accumulator slot
+        const int n = tile_n0(i) + h * 128 + q * 32 + lane;
+        const bool valid = n < p.N;
+        const uint32_t dcol = static_cast<uint32_t>(TA ? slot * BM + tok0 : b * 2 * BM + h * BM);
+        if (TA && nc == 0) {
+          // nothing to read: hand the slot back at once
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&dfree[slot]);
+        }
+        // A rolled loop over the 32-token chunks keeps the (unrolled) chunk
+        // body in the instruction cache: fully unrolled, the epilogue is
+        // straight-line code that runs once per tile and misses on every fetch.
+#pragma unroll 1
+        for (int c = 0; c < nc; ++c) {
+          float gsc = gs[0];
+          int xsc_ = xsum[0];
 #pragma unroll
-        for (int u = 1; u < kChunks; ++u)
-          if (c == u) {
-            gsc = gs[u];
-            xsc_ = xsum[u];
+          for (int w = 1; w < kChunks; ++w)
+            if (c == w) {
+              gsc = gs[w];
+              xsc_ = xsum[w];
+            }
+          uint32_t v[32];
+          tmem_ld_32x32b_x32(tmem + lane_base + dcol + static_cast<uint32_t>(32 * c), v);
+          tc_wait_ld();
+          if (TA && c + 1 == nc) {
+            // the last read of this slot has landed: the MMAs of the next
+            // tile may start while this warp stores
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&dfree[slot]);
           }
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem + lane_base + dcol + static_cast<uint32_t>(32 * c), v);
-        tc_wait_ld();
-        if (fast) {
-          // |acc| <= 128 K <= 2^22: conversions on the integer pipes (the
-          // conversion unit would otherwise bound the epilogue)
-          uint16_t* yb = static_cast<uint16_t*>(p.y) + static_cast<int64_t>(m0 + 32 * c) * p.N + n;
+          if (fast) {
+            // |acc| <= 128 K <= 2^22: conversions on the integer pipes (the
+            // conversion unit would otherwise bound the epilogue)
+            uint16_t* yb = static_cast<uint16_t*>(p.y) + static_cast<int64_t>(m0 + 32 * c) * p.N + n;
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const float gst = __shfl_sync(0xffffffffu, gsc, t);
-            const int xst = __shfl_sync(0xffffffffu, xsc_, t);
-            if (valid && m0 + 32 * c + t < p.M)
-              yb[static_cast<int64_t>(t) * p.N] =
-                  bf16_bits_rne(__fmul_rn(small_int_to_float(tc_dot<BITS>(v[t], xst)), gst));
-          }
-        } else {
+            for (int t = 0; t < 32; ++t) {
+              const float gst = __shfl_sync(0xffffffffu, gsc, t);
+              const int xst = __shfl_sync(0xffffffffu, xsc_, t);
+              if (valid && m0 + 32 * c + t < p.M)
+                yb[static_cast<int64_t>(t) * p.N] =
+                    bf16_bits_rne(__fmul_rn(small_int_to_float(tc_dot<BITS>(v[t], xst)), gst));
+            }
+          } else {
 #pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const float gst = __shfl_sync(0xffffffffu, gsc, t);
-            const int xst = __shfl_sync(0xffffffffu, xsc_, t);
-            const int m = m0 + 32 * c + t;
-            if (valid && m < p.M) {
-              const int acc = tc_dot<BITS>(v[t], xst);
-              const int64_t idx = static_cast<int64_t>(m) * p.N + n;
-              if (p.acc != nullptr) p.acc[idx] = acc;
-              if (p.y != nullptr) {
-                float o = __fmul_rn(__int2float_rn(acc), gst);
-                if (p.resid != nullptr) o = __fadd_rn(load_y(p.resid, p.y_dtype, idx), o);
-                store_y(p.y, p.y_dtype, idx, o);
+            for (int t = 0; t < 32; ++t) {
+              const float gst = __shfl_sync(0xffffffffu, gsc, t);
+              const int xst = __shfl_sync(0xffffffffu, xsc_, t);
+              const int m = m0 + 32 * c + t;
+              if (valid && m < p.M) {
+                const int acc = tc_dot<BITS>(v[t], xst);
+                const int64_t idx = static_cast<int64_t>(m) * p.N + n;
+                if (p.acc != nullptr) p.acc[idx] = acc;
+                if (p.y != nullptr) {
+                  float o = __fmul_rn(__int2float_rn(acc), gst);
+                  if (p.resid != nullptr) o = __fadd_rn(load_y(p.resid, p.y_dtype, idx), o);
+                  store_y(p.y, p.y_dtype, idx, o);
+                }
               }
             }
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&dfree[b]);
+      if (!TA) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dfree[b]);
+      }
     }
     pdl_launch_dependents();
   }

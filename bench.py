@@ -40,7 +40,7 @@ METRIC = "BitLinear decode GEMV HBM GB/s (% of peak); prefill GEMM int8 TOPS (% 
 # it stands (profiles/); set to None whenever the kernel changes.
 # Decode: 79.60 + 3.28 MB on the 4-layer stack, scaled by weight bytes to 30 layers.
 TRAFFIC_DECODE = round((79.602688e6 + 3.279872e6) * 597673800 / 79689840)
-TRAFFIC_PREFILL = None
+TRAFFIC_PREFILL = round(15.035648e6 + 4.606464e6)
 WORKLOAD = ("decode GEMV M=1 over the 2560x2560 / 2560x6912 / 6912x2560 BitLinear shapes, "
             "30-layer BitNet-b1.58-style stack (210 calls per token, 594.7 MB packed 2-bit weights)")
 NOMINAL_INT8_OVER_BF16 = 2.0        # dense int8 (as fp8) vs dense bf16, nominal B200 ratio
@@ -590,7 +590,7 @@ def run_prefill(args, dev, stream, bf16_peak, peak_src):
                    "l2": "flushed (256 MB write) before every timed iteration", "iters": args.prefill_iters},
         "value": round(ops / (full_ms * 1e-3) / 1e12, 2), "ms": round(full_ms, 4),
         "gemm_only_value": round(gemm_tops, 2), "gemm_only_ms": round(gemm_ms, 4),
-        "roofline": {"bound": "tensor", "kernel": "tc_gemm_persistent_kernel<128,8,2,2,TA> (tcgen05 kind::i8 TS form, 256x128 tiles, A expanded into TMEM, three rotating TMEM accumulator slots)", "achieved": round(gemm_tops, 2),
+        "roofline": {"bound": "tensor", "kernel": "tc_gemm_persistent_kernel<128,8,2,2> (tcgen05 kind::i8 TS form, 256x128 tiles, A expanded into TMEM, three rotating TMEM accumulator slots)", "achieved": round(gemm_tops, 2),
                      "peak": round(peak, 1), "unit": "TFLOP/s",
                      "frac": round(gemm_tops / peak, 4),
                      "peak_source": f"{peak_src} dense bf16 (burst) x {NOMINAL_INT8_OVER_BF16} nominal int8/bf16 ratio",

@@ -417,9 +417,9 @@ cudaError_t run_tc_t(const int8_t* xq, const TcParams& p, cudaStream_t st) {
 // Persistent tiles of 256 weight rows x BM tokens, one CTA per SM (the
 // shared-memory request keeps a second CTA off the SM: both want all 512
 // TMEM columns).
-template <int BM, int SS, int AS, int BITS, bool TA>
+template <int BM, int SS, int AS, int BITS>
 cudaError_t run_tp_t(const int8_t* xq, const TcParams& p, int sms, cudaStream_t st) {
-  static_assert(2 * tp_smem_bytes<BM, SS, AS, TA>() > 233472, "one CTA per SM");
+  static_assert(2 * tp_smem_bytes<BM, SS>() > 233472, "one CTA per SM");
   CUtensorMap map;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.K), static_cast<cuuint64_t>(p.M)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.K)};
@@ -429,8 +429,8 @@ cudaError_t run_tp_t(const int8_t* xq, const TcParams& p, int sms, cudaStream_t 
                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
-  auto k = tc_gemm_persistent_kernel<BM, SS, AS, BITS, TA>;
-  constexpr int smem = tp_smem_bytes<BM, SS, AS, TA>();
+  auto k = tc_gemm_persistent_kernel<BM, SS, AS, BITS>;
+  constexpr int smem = tp_smem_bytes<BM, SS>();
   cudaError_t e = allow_smem(k, smem);
   if (e != cudaSuccess) return e;
   const int64_t tiles = static_cast<int64_t>((p.N + kTpRows - 1) / kTpRows) * ((p.M + BM - 1) / BM);
@@ -446,7 +446,7 @@ cudaError_t run_tc_bits(const int8_t* xq, const TcParams& p, int sms, cudaStream
   if (p.M <= 16) return run_tc_t<16, 8, 4, BITS>(xq, p, st);
   if (p.M <= 32) return run_tc_t<32, 8, 4, BITS>(xq, p, st);
   if (p.M <= 64) return run_tc_t<64, 8, 4, BITS>(xq, p, st);
-  return run_tp_t<128, 8, 2, BITS, true>(xq, p, sms, st);
+  return run_tp_t<128, 8, 2, BITS>(xq, p, sms, st);
 }
 
 cudaError_t run_tc(const int8_t* xq, const TcParams& p, int sms, cudaStream_t st, int bits = 2) {

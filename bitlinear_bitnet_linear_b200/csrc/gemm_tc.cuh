@@ -323,56 +323,51 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
 // ---------------------------------------------------------------------------
 // Persistent variant (M > 64): one CTA per SM walks output tiles of 256
-// weight rows x BM tokens.  Each 128-wide K block feeds two M = 128 MMAs (the
-// two weight-row halves) that share one activation stage, halving the L2
-// traffic per MAC of a 128-row tile.  Both operands come from shared memory:
-// the converters expand the 2-bit codes to one unsigned byte per weight and
-// store them, 16 bytes at a time, in the 128-byte-swizzled K-major layout
-// that the TMA gives the activations.  All 512 TMEM columns hold two
-// accumulator buffers (2 x 2 halves x BM columns), so the epilogue of tile i
-// runs while the MMAs of tile i + 1 fill the other buffer.
+// weight rows x BM = 128 tokens.  Each 128-wide K block feeds two M = 128
+// MMAs (the two weight-row halves) that share one activation stage, halving
+// the L2 traffic per MAC of a 128-row tile.
+// A operand: the converters expand the 2-bit codes to one unsigned byte per
+// weight and write them to TMEM with tcgen05.st; the MMAs read A from there
+// (the TS form), so shared memory carries only the TMA-loaded activation
+// tiles (B).  With both operands in shared memory, one 128x128x32 int8 MMA
+// alone reads 8 KB in its 64-cycle slot, the SM's whole shared-memory
+// bandwidth, before any converter store or TMA write.
+// TMEM (512 columns): three accumulator slots of BM columns, then AS A
+// stages of 64 columns (weight-row half h at +32 h, 8 columns per 32-byte K
+// step).  Tile i accumulates its halves in slots 2i mod 3 and (2i + 1) mod
+// 3; tile i + 1 takes the third slot and tile i's first, so its MMAs start
+// as soon as the epilogue has read tile i's first half, while the epilogue
+// goes on with the second.
 // Roles (576 threads):
 //   warp 0        TMA producer, running ahead across tiles (SS stages)
 //   warp 1        TMEM allocator and single-thread MMA issuer
-//   warps 2..9    converters: one weight row per thread (AS stages)
-//   warps 10..17  epilogue: one weight row per thread (half (w-10)/4, TMEM
-//                 lane quadrant w % 4)
+//   warps 2..9    converters: one weight row per thread, rows of TMEM lane
+//                 quadrant w % 4 in half (w - 2) / 4 (a warp reaches only
+//                 lanes [32 (w % 4), 32 (w % 4) + 32))
+//   warps 10..17  epilogue: tokens [64 t, 64 t + 64), t = (w - 10) / 4, of
+//                 both halves, lane quadrant w % 4
 // Pipeline waits suspend in hardware (try_wait with a time hint), so warps
 // with nothing to do take no issue slots from the others; only the MMA
 // issuer, on the critical path, spins on its operand barriers.
 // Barriers: full/sempty (activation stages), afull/aempty (A stages; 256
-// converter arrivals), dfull[b] (all MMAs of a tile done), dfree[b] (8
-// epilogue warps done reading buffer b), mdone (every MMA issued has
-// completed, before TMEM is freed).
-//
-// TA = true keeps the expanded codes out of shared memory: the converters
-// write them to TMEM with tcgen05.st and the MMAs take A from there (the TS
-// form), so shared memory carries only the activation tiles.  TMEM then
-// holds three accumulator slots of BM columns and AS A stages of 64 columns
-// (two halves of 32).  Tile i accumulates its weight-row halves in slots
-// 2i mod 3 and (2i + 1) mod 3; tile i + 1 takes the third slot and tile i's
-// first, so its MMAs start as soon as the epilogue has read tile i's first
-// half (dfree[s]: slot s read by all 8 epilogue warps, which drain the two
-// halves in order, each warp 64 tokens of one TMEM lane quadrant).
+// converter arrivals), dfull (all MMAs of a tile done), dfree[s] (8 epilogue
+// warps done reading slot s), mdone (every MMA issued has completed, before
+// TMEM is freed).
 // ---------------------------------------------------------------------------
 constexpr int kTpRows = 256;
 constexpr int kTpThreads = 18 * 32;
-constexpr int kTpAStage = kTpRows * kTcBK;     // 32 KB of expanded codes per K block
 
-template <int BM, int SS, int AS, bool TA = false>
+template <int BM, int SS>
 __host__ __device__ constexpr int tp_smem_bytes() {
-  return 1024 /* alignment slack */ + SS * BM * kTcBK + (TA ? 0 : AS * kTpAStage) + 1024 /* barriers, flags */;
+  return 1024 /* alignment slack */ + SS * BM * kTcBK + 1024 /* barriers, flags */;
 }
 
-template <int BM, int SS, int AS, int BITS = 2, bool TA = false>
+template <int BM, int SS, int AS, int BITS = 2>
 __global__ void __launch_bounds__(kTpThreads, 1)
     tc_gemm_persistent_kernel(const __grid_constant__ CUtensorMap tmap_x, const TcParams p) {
-  static_assert(BM == 128 && (!TA || 3 * BM + 64 * AS <= 512),
-                "the accumulators (and the TMEM A stages) fit the 512 TMEM columns");
+  static_assert(BM == 128 && 3 * BM + 64 * AS <= 512, "the accumulator slots and A stages fit 512 TMEM columns");
   constexpr uint32_t kCols = 512;
-  constexpr int kDB = TA ? 1 : 2;                      // tile-completion barriers in turn
-  constexpr uint32_t kACol0 = 3 * BM;                  // TA: A stage a at [3 BM + 64 a, 3 BM + 64 a + 64)
-  constexpr int kASmem = TA ? 0 : kTpAStage;           // shared-memory bytes of one A stage
+  constexpr uint32_t kACol0 = 3 * BM;                  // A stage a at [3 BM + 64 a, 3 BM + 64 a + 64)
   constexpr uint32_t kStageBytes = BM * kTcBK;
   constexpr uint32_t kIdesc = idesc_i8_us(kTcBN, BM);
   constexpr int kPD = 4;                               // converter prefetch depth (K blocks)
@@ -380,13 +375,12 @@ __global__ void __launch_bounds__(kTpThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = smem;
-  uint8_t* as = smem + SS * kStageBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(as + AS * kASmem);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + SS * kStageBytes);
   uint64_t* sempty = full + SS;
   uint64_t* afull = sempty + SS;
   uint64_t* aempty = afull + AS;
   uint64_t* dfull = aempty + AS;
-  uint64_t* dfree = dfull + 2;
+  uint64_t* dfree = dfull + 1;
   uint64_t* mdone = dfree + 3;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(mdone + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
@@ -411,8 +405,8 @@ __global__ void __launch_bounds__(kTpThreads, 1)
       mbar_init(&afull[a], 256);
       mbar_init(&aempty[a], 1);
     }
-    for (int b = 0; b < 2; ++b) mbar_init(&dfull[b], 1);
-    for (int b = 0; b < 3; ++b) mbar_init(&dfree[b], 8);
+    mbar_init(dfull, 1);
+    for (int s = 0; s < 3; ++s) mbar_init(&dfree[s], 8);
     mbar_init(mdone, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -462,33 +456,20 @@ __global__ void __launch_bounds__(kTpThreads, 1)
     if (lane == 0) {
       bool ok = true;
       int g = 0;
-      uint32_t slot_par = 0;   // TA: bit s = parity of the uses of slot s so far
+      uint32_t slot_par = 0;   // bit s = parity of the uses of slot s so far
       for (int i = 0; i < my_tiles && ok; ++i) {
-        const int b = i % kDB;
-        uint32_t d0, d1;         // accumulators of the two weight-row halves
-        if constexpr (TA) {
-          const int s0 = (2 * i) % 3, s1 = (2 * i + 1) % 3;
-          // the epilogue has read what earlier tiles left in both slots
-          if (!mbar_wait_sleep(&dfree[s0], ((slot_par >> s0) & 1u) ^ 1u, p.limit_ns, abort_flag) ||
-              !mbar_wait_sleep(&dfree[s1], ((slot_par >> s1) & 1u) ^ 1u, p.limit_ns, abort_flag)) {
-            if (!*abort_flag) fail(0x312u);
-            ok = false;
-            break;
-          }
-          slot_par ^= (1u << s0) | (1u << s1);
-          d0 = tmem + static_cast<uint32_t>(s0 * BM);
-          d1 = tmem + static_cast<uint32_t>(s1 * BM);
-        } else {
-          // the epilogue has read what the tile before last left in buffer b
-          if (!mbar_wait_sleep(&dfree[b], ((i >> 1) & 1) ^ 1u, p.limit_ns, abort_flag)) {
-            if (!*abort_flag) fail(0x312u);
-            ok = false;
-            break;
-          }
-          d0 = tmem + static_cast<uint32_t>(b * 2 * BM);
-          d1 = d0 + BM;
+        const int s0 = (2 * i) % 3, s1 = (2 * i + 1) % 3;
+        // the epilogue has read what earlier tiles left in both slots
+        if (!mbar_wait_sleep(&dfree[s0], ((slot_par >> s0) & 1u) ^ 1u, p.limit_ns, abort_flag) ||
+            !mbar_wait_sleep(&dfree[s1], ((slot_par >> s1) & 1u) ^ 1u, p.limit_ns, abort_flag)) {
+          if (!*abort_flag) fail(0x312u);
+          ok = false;
+          break;
         }
+        slot_par ^= (1u << s0) | (1u << s1);
         tc_fence_after();
+        const uint32_t d0 = tmem + static_cast<uint32_t>(s0 * BM);   // weight-row half 0
+        const uint32_t d1 = tmem + static_cast<uint32_t>(s1 * BM);   // weight-row half 1
         for (int kb = 0; kb < KB; ++kb, ++g) {
           const int s = g % SS;
           const int a = g % AS;
@@ -501,30 +482,18 @@ __global__ void __launch_bounds__(kTpThreads, 1)
           }
           tc_fence_after();
           const uint64_t bdesc = smem_desc_k_sw128(smem_u32(xs + s * kStageBytes));
-          if constexpr (TA) {
-            const uint32_t a0 = tmem + kACol0 + 64u * static_cast<uint32_t>(a);
+          const uint32_t a0 = tmem + kACol0 + 64u * static_cast<uint32_t>(a);
 #pragma unroll
-            for (int j = 0; j < kTcBK / 32; ++j) {
-              // K step of 32 bytes: 8 TMEM columns of A, 32 B of the B descriptor (>> 4 = 2)
-              const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
-              tc_mma_i8_ts(d0, a0 + 8u * j, bdesc + 2ull * j, kIdesc, acc);
-              tc_mma_i8_ts(d1, a0 + 32u + 8u * j, bdesc + 2ull * j, kIdesc, acc);
-            }
-          } else {
-            const uint64_t adesc0 = smem_desc_k_sw128(smem_u32(as + a * kTpAStage));
-            const uint64_t adesc1 = smem_desc_k_sw128(smem_u32(as + a * kTpAStage + kTpAStage / 2));
-#pragma unroll
-            for (int j = 0; j < kTcBK / 32; ++j) {
-              // K step of 32 bytes: advance both descriptors' start address by 32 B (>> 4 = 2)
-              const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
-              tc_mma_i8_ss(d0, adesc0 + 2ull * j, bdesc + 2ull * j, kIdesc, acc);
-              tc_mma_i8_ss(d1, adesc1 + 2ull * j, bdesc + 2ull * j, kIdesc, acc);
-            }
+          for (int j = 0; j < kTcBK / 32; ++j) {
+            // K step of 32 bytes: 8 TMEM columns of A, 32 B of the B descriptor (>> 4 = 2)
+            const uint32_t acc = (kb | j) != 0 ? 1u : 0u;
+            tc_mma_i8_ts(d0, a0 + 8u * j, bdesc + 2ull * j, kIdesc, acc);
+            tc_mma_i8_ts(d1, a0 + 32u + 8u * j, bdesc + 2ull * j, kIdesc, acc);
           }
           tc_commit(&sempty[s]);
           tc_commit(&aempty[a]);
         }
-        if (ok) tc_commit(&dfull[b]);
+        if (ok) tc_commit(dfull);
       }
       // every MMA issued has completed before TMEM can be freed
       tc_commit(mdone);
@@ -533,12 +502,9 @@ __global__ void __launch_bounds__(kTpThreads, 1)
     pdl_launch_dependents();
   } else if (warp < 10) {
     // ------------------------------------------------------------ converters
-    // A row of the 256-row tile.  TA: warp w may only reach TMEM lanes
-    // [32 (w % 4), 32 (w % 4) + 32), so it takes rows of lane quadrant w % 4
-    // in half (w - 2) / 4.
-    const int row = TA ? ((warp - 2) >> 2) * 128 + (warp & 3) * 32 + lane : (warp - 2) * 32 + lane;
-    const uint32_t a_lane_col = (static_cast<uint32_t>((warp & 3) * 32) << 16) + kACol0 +
-                                32u * static_cast<uint32_t>((warp - 2) >> 2);
+    const int h = (warp - 2) >> 2;                     // weight-row half
+    const int row = h * 128 + (warp & 3) * 32 + lane;  // A row of the 256-row tile
+    const uint32_t a_lane_col = (static_cast<uint32_t>((warp & 3) * 32) << 16) + kACol0 + 32u * h;
     const int rowbytes = p.K * BITS / 8;
     const int total = my_tiles * KB;
     uint32_t wb[kPD][8];
@@ -552,8 +518,6 @@ __global__ void __launch_bounds__(kTpThreads, 1)
 #pragma unroll
     for (int j = 0; j < kPD; ++j)
       if (j < total) load(j, wb[j]);
-    // 16-byte chunk c of this row sits at chunk c ^ (row % 8) (128-byte swizzle)
-    const uint32_t swz = static_cast<uint32_t>(row & 7);
     bool ok = true;
     for (int g0 = 0; g0 < total && ok; g0 += kPD) {
 #pragma unroll
@@ -565,37 +529,25 @@ __global__ void __launch_bounds__(kTpThreads, 1)
             if (!*abort_flag) fail(0x314u);
             ok = false;
           }
-          if constexpr (TA) {
-            // tcgen05.st is warp-collective: the warp goes on only together
-            // (the waits return together unless aborting)
-            if (__all_sync(0xffffffffu, ok)) {
-              uint32_t codes[32];
+          // tcgen05.st is warp-collective: the warp goes on only together
+          // (the waits return together unless aborting)
+          if (__all_sync(0xffffffffu, ok)) {
+            uint32_t codes[32];
 #pragma unroll
-              for (int c = 0; c < 8; ++c) {
-                const uint4 c4 = tc_expand_chunk<BITS>(wb[j], c);
-                codes[4 * c + 0] = c4.x;
-                codes[4 * c + 1] = c4.y;
-                codes[4 * c + 2] = c4.z;
-                codes[4 * c + 3] = c4.w;
-              }
-              tmem_st_32x32b_x32(tmem + a_lane_col + 64u * static_cast<uint32_t>(a), codes);
-              tc_wait_st();
-              tc_fence_before();
-              mbar_arrive(&afull[a]);
-              if (g + kPD < total) load(g + kPD, wb[j]);
-            } else {
-              ok = false;
+            for (int c = 0; c < 8; ++c) {   // chunk c: weights 16c .. 16c + 15 of the K block
+              const uint4 c4 = tc_expand_chunk<BITS>(wb[j], c);
+              codes[4 * c + 0] = c4.x;
+              codes[4 * c + 1] = c4.y;
+              codes[4 * c + 2] = c4.z;
+              codes[4 * c + 3] = c4.w;
             }
-          } else if (ok) {
-            uint8_t* arow = as + a * kTpAStage + row * kTcBK;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)   // chunk c: weights 16c .. 16c + 15 of the K block
-              *reinterpret_cast<uint4*>(arow + ((static_cast<uint32_t>(c) ^ swz) << 4)) =
-                  tc_expand_chunk<BITS>(wb[j], c);
-            // the tensor core reads these bytes through the async proxy
-            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            tmem_st_32x32b_x32(tmem + a_lane_col + 64u * static_cast<uint32_t>(a), codes);
+            tc_wait_st();
+            tc_fence_before();
             mbar_arrive(&afull[a]);
             if (g + kPD < total) load(g + kPD, wb[j]);
+          } else {
+            ok = false;
           }
         }
       }
@@ -603,16 +555,10 @@ __global__ void __launch_bounds__(kTpThreads, 1)
     pdl_launch_dependents();
   } else {
     // ------------------------------------------------------------ epilogue
-    // Shared-memory A: warp w drains all BM tokens of weight-row half
-    // (w - 10) / 4.  TMEM A: warp w drains tokens [64 t, 64 t + 64),
-    // t = (w - 10) / 4, of both halves, the first half's slot first.
-    // Either way the warp reads TMEM lane quadrant w % 4.
-    const int q = warp & 3;
-    const int h_own = TA ? 0 : (warp - 10) >> 2;
-    const int tok0 = TA ? ((warp - 10) >> 2) * 64 : 0;
+    const int q = warp & 3;                     // TMEM lane quadrant
+    const int tok0 = ((warp - 10) >> 2) * 64;   // first token of this warp in the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    constexpr int kChunks = (TA ? 64 : BM) / 32;
-    constexpr int kHalves = TA ? 2 : 1;
+    constexpr int kChunks = 2;                  // 64 tokens in chunks of 32
     const bool fast = p.y != nullptr && p.acc == nullptr && p.resid == nullptr && p.y_dtype == BITNET_BF16 &&
                       p.K <= 32768;
     pdl_wait();   // token scales and sums come from the previous kernel
@@ -620,8 +566,6 @@ __global__ void __launch_bounds__(kTpThreads, 1)
     const float* __restrict__ xsc = p.x_scale;
     const int32_t* __restrict__ xsm = p.x_sum;
     for (int i = 0; i < my_tiles; ++i) {
-      const int b = i % kDB;
-      const int u = i / kDB;   // earlier uses of barrier b
       const int m0 = tile_m0(i) + tok0;   // this warp's first token
       // chunks of 32 tokens holding tokens below M (warp-uniform)
       const int nc = min(kChunks, (max(0, p.M - m0) + 31) / 32);
@@ -639,20 +583,19 @@ __global__ void __launch_bounds__(kTpThreads, 1)
           xsum[c] = __ldg(xsm + mi);
         }
       }
-      const bool got = mbar_wait_sleep(&dfull[b], u & 1, p.limit_ns, abort_flag);
+      const bool got = mbar_wait_sleep(dfull, i & 1, p.limit_ns, abort_flag);
       if (!got && !*abort_flag) fail(0x315u);
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       if (i + 1 == my_tiles) pdl_launch_dependents();
 #pragma unroll 1
-      for (int hh = 0; hh < kHalves; ++hh) {
-        const int h = TA ? hh : h_own;                 // weight-row half
-        const int slot = TA ? (2 * i + hh) % 3 : 0;    // TA: its accumulator slot
+      for (int h = 0; h < 2; ++h) {                    // weight-row half, its slot
+        const int slot = (2 * i + h) % 3;
         const int n = tile_n0(i) + h * 128 + q * 32 + lane;
         const bool valid = n < p.N;
-        const uint32_t dcol = static_cast<uint32_t>(TA ? slot * BM + tok0 : b * 2 * BM + h * BM);
-        if (TA && nc == 0) {
-          // nothing to read: hand the slot back at once
+        const uint32_t dcol = static_cast<uint32_t>(slot * BM + tok0);
+        if (nc == 0) {
+          // no token of this warp in the tile: hand the slot back at once
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&dfree[slot]);
@@ -662,18 +605,12 @@ __global__ void __launch_bounds__(kTpThreads, 1)
         // straight-line code that runs once per tile and misses on every fetch.
 #pragma unroll 1
         for (int c = 0; c < nc; ++c) {
-          float gsc = gs[0];
-          int xsc_ = xsum[0];
-#pragma unroll
-          for (int w = 1; w < kChunks; ++w)
-            if (c == w) {
-              gsc = gs[w];
-              xsc_ = xsum[w];
-            }
+          const float gsc = c == 0 ? gs[0] : gs[1];
+          const int xsc_ = c == 0 ? xsum[0] : xsum[1];
           uint32_t v[32];
           tmem_ld_32x32b_x32(tmem + lane_base + dcol + static_cast<uint32_t>(32 * c), v);
           tc_wait_ld();
-          if (TA && c + 1 == nc) {
+          if (c + 1 == nc) {
             // the last read of this slot has landed: the MMAs of the next
             // tile may start while this warp stores
             tc_fence_before();
@@ -711,11 +648,6 @@ __global__ void __launch_bounds__(kTpThreads, 1)
             }
           }
         }
-      }
-      if (!TA) {
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&dfree[b]);
       }
     }
     pdl_launch_dependents();

@@ -392,6 +392,17 @@ def run_ours(args):
                       "grouped launch per token (bitnet_linear_grouped_t3), digits decoded in registers"}
         del t3_graph, t3_call, t3_packed
 
+    # ---- single-matrix HBM gates: each shape at M = 1 over a pool of distinct
+    # weight copies (together well beyond L2), as separate launches and as
+    # one grouped launch.  A failure here is reported in its own key. -------
+    gates = None
+    if not args.no_chain:
+        try:
+            gates = hbm_gate_legs(bn, synthetic, dev, stream, capture, time_graph, world, gains)
+        except Exception as e:   # noqa: BLE001 - the headline line must still print
+            gates = {"error": repr(e)[:300]}
+        torch.cuda.synchronize()
+
     # ---- e2e: host buffers, through the public API, no graph ----------------
     e2e = None
     if not args.no_e2e:
@@ -508,11 +519,68 @@ def run_ours(args):
         out["b1_decode"] = b1
     if t3 is not None:
         out["t3_decode"] = t3
+    if gates is not None:
+        out["hbm_gates"] = gates
     if prefill is not None:
         out["prefill"] = prefill
     if cpu is not None:
         out["cpu_baseline"] = cpu
     return out
+
+
+L2_BYTES = 126 * 2 ** 20
+GATE_SHAPES = [(8192, 28672), (28672, 8192), (2560, 2560), (2560, 6912), (6912, 2560)]   # (K, N)
+
+
+def hbm_gate_legs(bn, synthetic, dev, stream, capture, time_graph, world, gains):
+    """Decode (M = 1) over one shape at a time.  Each shape gets a pool of
+    distinct copies of one packed matrix, at least 3x L2 in total (at most
+    240 copies), with its own bf16 activation row and output per copy:
+    - single: one bitnet_linear launch per copy, in stream order, one CUDA
+      graph per pass over the pool;
+    - grouped: the whole pool as one bitnet_linear_grouped launch.
+    Bytes per call: N K / 4 + 2 K + 2 N + 4."""
+    import torch
+    res = []
+    for K, N in GATE_SHAPES:
+        wbytes = N * K // 4
+        copies = int(min(240, max(8, -(-3 * L2_BYTES // wbytes))))
+        gen = torch.Generator(device=dev).manual_seed(7000 + K + N)
+        with torch.cuda.stream(stream):
+            W = torch.randn((N, K), generator=gen, device=dev, dtype=torch.float32) * synthetic.W_SIGMA
+            Wq, g = bn.bitnet_quant_weights(W)
+            Wp0 = bn.bitnet_pack(Wq)
+            del W, Wq
+            pool = [Wp0.clone() for _ in range(copies)]
+        torch.cuda.synchronize()
+        del Wp0
+        gain = gains[K] if K in gains else synthetic.unit_gain(K).to(dev)
+        xs = [synthetic.activations(1, K, seed=8000 + i, dtype=torch.bfloat16).to(dev) for i in range(copies)]
+        ys = [torch.empty((1, N), dtype=torch.bfloat16, device=dev) for _ in range(copies)]
+        ws = bn.new_workspace(bn.bitnet_workspace_bytes(1, K, N), dev)
+        call_bytes = wbytes + 2 * K + 2 * N + 4
+
+        def single():
+            for Wp, x, y in zip(pool, xs, ys):
+                bn.bitnet_linear(x, Wp, g, N=N, rms_gain=gain, rms_eps=1e-5, y=y, ws=ws)
+
+        grouped = bn.GroupedCall([(x, Wp, g, gain, y) for Wp, x, y in zip(pool, xs, ys)], rms_eps=1e-5, ws=ws)
+        entry = {"K": K, "N": N, "copies": copies, "pool_mb": round(copies * wbytes / 1e6, 1),
+                 "bytes_per_call": call_bytes}
+        for name, fn in (("single", single), ("grouped", grouped)):
+            gr = capture(fn)
+            ms, ms_max, _ = time_graph(gr, 20, 3)
+            assert bn.bitnet_get_error(ws) == 0
+            entry[name] = {"value": round(world * copies * call_bytes / (ms_max * 1e-3) / 1e9, 2), "unit": "GB/s",
+                           "us_per_call": round(ms_max * 1e3 / copies, 3)}
+            del gr
+        res.append(entry)
+        del pool, xs, ys, grouped
+        torch.cuda.synchronize()
+    return {"what": "M = 1 BitLinear (bf16 x, unit RMSNorm gain, bf16 y) per shape over a pool of distinct "
+                    "weight copies of at least 3x L2; single = one bitnet_linear launch per call in stream "
+                    "order, grouped = the pool as one bitnet_linear_grouped launch; CUDA graphs, 20 passes",
+            "shapes": res}
 
 
 def run_prefill(args, dev, stream, bf16_peak, peak_src):

@@ -392,17 +392,6 @@ def run_ours(args):
                       "grouped launch per token (bitnet_linear_grouped_t3), digits decoded in registers"}
         del t3_graph, t3_call, t3_packed
 
-    # ---- single-matrix HBM gates: each shape at M = 1 over a pool of distinct
-    # weight copies (together well beyond L2), as separate launches and as
-    # one grouped launch.  A failure here is reported in its own key. -------
-    gates = None
-    if not args.no_chain:
-        try:
-            gates = hbm_gate_legs(bn, synthetic, dev, stream, capture, time_graph, world, gains)
-        except Exception as e:   # noqa: BLE001 - the headline line must still print
-            gates = {"error": repr(e)[:300]}
-        torch.cuda.synchronize()
-
     # ---- e2e: host buffers, through the public API, no graph ----------------
     e2e = None
     if not args.no_e2e:
@@ -476,6 +465,18 @@ def run_ours(args):
     cpu = None
     if not args.no_cpu_baseline and world == 1 and rank == 0:
         cpu = cpu_baseline(layers_sample=1)
+
+    # ---- single-matrix HBM gates: each shape at M = 1 over a pool of distinct
+    # weight copies (together well beyond L2), as separate launches and as
+    # one grouped launch.  Last, so that nothing else depends on it; a
+    # failure here is reported in its own key. ------------------------------
+    gates = None
+    if not args.no_chain:
+        try:
+            gates = hbm_gate_legs(bn, synthetic, dev, stream, capture, time_graph, world, gains)
+            torch.cuda.synchronize()
+        except Exception as e:   # noqa: BLE001 - the headline line must still print
+            gates = {"error": repr(e)[:300]}
 
     del graph, graph1
     if world > 1:

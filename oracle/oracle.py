@@ -17,8 +17,11 @@ import subprocess
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "bitnet_oracle.c")
-_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+# BITNET_ORACLE_SRC / BITNET_ORACLE_LIB point the module at another copy of
+# the C source and its build: the mutation tests plant a mistake in a copy
+# and check that the pins reject it.
+_SRC = os.environ.get("BITNET_ORACLE_SRC") or os.path.join(_HERE, "bitnet_oracle.c")
+_LIB_PATH = os.environ.get("BITNET_ORACLE_LIB") or os.path.join(_HERE, "liboracle.so")
 
 # The activation floor that guards an all-zero row (the pages are silent).
 FLOOR_EPS = 1e-5

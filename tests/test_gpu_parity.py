@@ -173,6 +173,9 @@ ACC_CASES = [
     (129, 1024, 1000), (257, 2560, 384), (300, 64, 200),
     # 512 tokens and more: tiles of 128 weight rows x 256 tokens, ragged in both
     (512, 256, 128), (600, 1024, 1000), (777, 272, 129),
+    # the persistent kernel's edges: one token over the small-kernel limit, a
+    # single weight row, K below one 128-wide block (scalar weight loads)
+    (65, 2560, 7), (70, 16, 1), (1000, 32, 2),
 ]
 
 

@@ -469,9 +469,10 @@ def run_ours(args):
     # ---- single-matrix HBM gates: each shape at M = 1 over a pool of distinct
     # weight copies (together well beyond L2), as separate launches and as
     # one grouped launch.  Last, so that nothing else depends on it; a
-    # failure here is reported in its own key. ------------------------------
+    # failure here is reported in its own key.  One GPU only: a failure on
+    # one rank must not leave the ranks' collectives out of step. -----------
     gates = None
-    if not args.no_chain:
+    if not args.no_chain and world == 1:
         try:
             gates = hbm_gate_legs(bn, synthetic, dev, stream, capture, time_graph, world, gains)
             torch.cuda.synchronize()

@@ -740,10 +740,16 @@ static bitnet_status linear_impl(const void* x, int x_dtype, const int8_t* xq_in
     }
     cudaError_t e = (s == BITNET_OK) ? run_stream<kStreamSmallP>(*pl, st) : cudaSuccess;
     delete pl;
-    if (s != BITNET_OK) return s;
-    return launch_result(e);
-  }
-  if (use_gemv) {
+    // A very long row (the activations plus one packed row per ring slot
+    // beyond shared memory) has no streaming plan; the automatic choice then
+    // takes the tensor-core path, which handles any K.  Base-3 weights have
+    // no tensor-core path.
+    const bool to_tc = s == BITNET_ERR_UNSUPPORTED && path == BITNET_PATH_AUTO && bits != 3;
+    if (!to_tc) {
+      if (s != BITNET_OK) return s;
+      return launch_result(e);
+    }
+  } else if (use_gemv) {
     GemvParams& p = gp.p;
     p.x = x;
     p.x_dtype = x_dtype;

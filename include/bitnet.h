@@ -172,8 +172,9 @@ bitnet_status bitnet_unpack_b1(const uint8_t *Wp, int64_t N, int64_t K, int8_t *
  *   acc[m,n] = sum_k x_q[m,k] * W_b[n,k] = 2 sum_{W_b = +1} x_q - sum_k x_q
  *   y[m,n]   = (float)acc[m,n] * (beta * s_x[m]).
  * K % 128 == 0 (else BITNET_ERR_SHAPE).  M = 1 runs the fused streaming
- * GEMV; larger M the quantiser then the tensor-core GEMM.  Wp: [N, K/8]
- * (bitnet_pack_b1).  ws: bitnet_workspace_bytes(M, K, N) bytes. */
+ * GEMV (up to K = 79872; beyond, the tensor-core path); larger M the
+ * quantiser then the tensor-core GEMM.  Wp: [N, K/8] (bitnet_pack_b1).
+ * ws: bitnet_workspace_bytes(M, K, N) bytes. */
 bitnet_status bitnet_linear_b1(const void *x, int x_dtype, int64_t M, int64_t K,
                                const uint8_t *Wp, int64_t N, const float *beta,
                                const float *rms_gain, float rms_eps,
@@ -206,8 +207,9 @@ bitnet_status bitnet_unpack_t3(const uint8_t *Wp, int64_t N, int64_t K, int8_t *
 
 /* BitLinear forward of ONE token (x [1, K]) with base-3 packed weights:
  * y[n] exactly as bitnet_linear would give with the same ternary weights.
- * The streaming GEMV decodes the base-3 digits in registers.  ws:
- * bitnet_workspace_bytes(1, K, N) bytes. */
+ * The streaming GEMV decodes the base-3 digits in registers; it bounds K
+ * at 57600 (BITNET_ERR_UNSUPPORTED beyond: this format has no tensor-core
+ * path).  ws: bitnet_workspace_bytes(1, K, N) bytes. */
 bitnet_status bitnet_linear_t3(const void *x, int x_dtype, int64_t K,
                                const uint8_t *Wp, int64_t N, const float *gamma,
                                const float *rms_gain, float rms_eps,
@@ -249,7 +251,11 @@ bitnet_status bitnet_quant_act(const void *x, int x_dtype, int64_t M, int64_t K,
  * Wp: [N, K/4] packed weights (bitnet_pack).  gamma: device binary32.
  * y: [M, N] of y_dtype.  ws: bitnet_workspace_bytes(M, K, N) bytes.
  * Small M runs one fused kernel (quantise + GEMV); larger M runs the
- * quantiser then the tensor-core GEMM. */
+ * quantiser then the tensor-core GEMM.  The fused kernel holds the
+ * quantised activations and one packed weight row per ring slot in shared
+ * memory, which bounds K at 48128 (M = 1), 39936 (M = 2) and 29696
+ * (M = 3, 4) for 2-bit weights; beyond that the automatic choice takes the
+ * tensor-core path, which has no K bound. */
 bitnet_status bitnet_linear(const void *x, int x_dtype, int64_t M, int64_t K,
                             const uint8_t *Wp, int64_t N, const float *gamma,
                             const float *rms_gain, float rms_eps,
@@ -257,7 +263,8 @@ bitnet_status bitnet_linear(const void *x, int x_dtype, int64_t M, int64_t K,
                             bitnet_stream_t stream);
 
 /* bitnet_linear with an explicit path (BITNET_PATH_*).  BITNET_PATH_GEMV
- * with M > 4 returns BITNET_ERR_UNSUPPORTED. */
+ * with M > 4, or with K beyond the fused kernel's bound (see
+ * bitnet_linear), returns BITNET_ERR_UNSUPPORTED. */
 bitnet_status bitnet_linear_ex(const void *x, int x_dtype, int64_t M, int64_t K,
                                const uint8_t *Wp, int64_t N, const float *gamma,
                                const float *rms_gain, float rms_eps,
@@ -321,8 +328,10 @@ typedef struct bitnet_gemv_problem {
  * layers of one block share their input).  The problems' outputs must not
  * overlap each other's inputs.
  * problems: host array of `count` entries (1 <= count <= 256), read during
- * the call only.  Every K must be a multiple of 64.  ws: at least
- * bitnet_workspace_bytes(1, 16, 1) bytes (status word only). */
+ * the call only.  Every K must be a multiple of 64, and the largest K at
+ * most the fused kernel's bound (bitnet_linear: 48128 at M = 1, 39936 at
+ * M = 2, 29696 at M = 3, 4); otherwise BITNET_ERR_UNSUPPORTED.  ws: at
+ * least bitnet_workspace_bytes(1, 16, 1) bytes (status word only). */
 bitnet_status bitnet_linear_grouped(const bitnet_gemv_problem *problems, int count, int64_t M,
                                     int x_dtype, float rms_eps, int y_dtype,
                                     void *ws, size_t ws_bytes, bitnet_stream_t stream);
@@ -349,14 +358,15 @@ bitnet_status bitnet_quant_weights_noalloc(const float *W, int64_t N, int64_t K,
                                            int8_t *Wq, float *gamma, bitnet_stream_t stream);
 
 /* bitnet_linear_grouped for BitNet b1 weights (bitnet_pack_b1, Wp [N, K/8],
- * gamma = beta), one token (M = 1), K % 128 == 0: each problem is computed
- * exactly as bitnet_linear_b1. */
+ * gamma = beta), one token (M = 1), K % 128 == 0, K <= 79872: each problem
+ * is computed exactly as bitnet_linear_b1. */
 bitnet_status bitnet_linear_grouped_b1(const bitnet_gemv_problem *problems, int count, int x_dtype,
                                        float rms_eps, int y_dtype, void *ws, size_t ws_bytes,
                                        bitnet_stream_t stream);
 
 /* bitnet_linear_grouped for base-3 packed weights (bitnet_pack_t3), one
- * token (M = 1): each problem is computed exactly as bitnet_linear_t3. */
+ * token (M = 1), K <= 57600: each problem is computed exactly as
+ * bitnet_linear_t3. */
 bitnet_status bitnet_linear_grouped_t3(const bitnet_gemv_problem *problems, int count, int x_dtype,
                                        float rms_eps, int y_dtype, void *ws, size_t ws_bytes,
                                        bitnet_stream_t stream);

@@ -88,6 +88,18 @@ def test_linear_b1_matches_oracle(M, K, N, with_gain):
     assert np.array_equal(y16.cpu().view(torch.int16).numpy().astype(np.uint16), oracle.to_bf16_bits(y_ref))
 
 
+def test_linear_b1_long_row_takes_tensor_core_path():
+    """M = 1 with K beyond the fused GEMV's bound for 1-bit rows (79872)."""
+    M, K, N = 1, 81920, 24
+    x = synthetic.activations(M, K, seed=321, dtype=torch.bfloat16)
+    Wb, beta, Wp, beta_d = b1_weights(N, K, seed=654)
+    xq, sc, _ = oracle.quant_act(x.float().numpy())
+    y_ref = oracle.output(oracle.linear_i32(xq, Wb), beta, sc)
+    y = bn.bitnet_linear_b1(x.to(DEV), Wp, beta_d, N=N, y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert np.array_equal(y.cpu().numpy(), y_ref)
+
+
 def test_linear_b1_rejects_k_not_multiple_of_128():
     x = torch.zeros(1, 192, dtype=torch.bfloat16, device=DEV)
     Wp = torch.zeros(8, 24, dtype=torch.uint8, device=DEV)

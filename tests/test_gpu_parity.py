@@ -269,6 +269,24 @@ def test_large_shapes_sampled(M, K, N):
     _sampled_check(M, K, N, seed=900 + M + K, norm=False, sample_rows=2)
 
 
+# K beyond the fused GEMV's shared-memory bound (48128 at M = 1, 39936 at
+# M = 2, 29696 at M = 3, 4): the automatic path takes the tensor-core GEMM,
+# the forced GEMV path reports UNSUPPORTED
+@pytest.mark.parametrize("M,K", [(1, 53248), (1, 57344), (2, 45056), (4, 32768)])
+def test_long_rows_take_tensor_core_path(M, K):
+    N = 40
+    _, Wq, g, Wp, x = _prep(M, K, N, seed=M + K)
+    y_ref, *_ = oracle.bitlinear(xf32(x), Wq, g)
+    Wp_d = torch.from_numpy(Wp).to(DEV)
+    gd = torch.tensor([g], dtype=torch.float32, device=DEV)
+    y = bn.bitnet_linear(x.to(DEV), Wp_d, gd, y_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert np.array_equal(to_np(y), y_ref)   # no gain: the same IEEE operations, bit-exact
+    with pytest.raises(bn.BitnetError) as ei:
+        bn.bitnet_linear(x.to(DEV), Wp_d, gd, path=bn.PATH_GEMV)
+    assert ei.value.status == 5
+
+
 # ---------------------------------------------------------------------------
 # errors and the watchdog
 # ---------------------------------------------------------------------------

@@ -523,6 +523,13 @@ def run_ours(args):
         out["t3_decode"] = t3
     if gates is not None:
         out["hbm_gates"] = gates
+    # every HBM-bound leg against the same measured copy bandwidth, per GPU
+    for key in ("decode_chain", "ffn_chain", "b1_decode", "t3_decode"):
+        if key in out:
+            out[key]["frac_of_hbm_peak"] = round(out[key]["value"] / world / hbm_peak, 4)
+    for e in (gates or {}).get("shapes", []):
+        for form in ("single", "grouped"):
+            e[form]["frac_of_hbm_peak"] = round(e[form]["value"] / world / hbm_peak, 4)
     if prefill is not None:
         out["prefill"] = prefill
     if cpu is not None:

@@ -116,6 +116,9 @@ def _ptr(t):
         return None
     if not t.is_cuda:
         raise ValueError("tensor must be on a CUDA device")
+    if t.device.index != torch.cuda.current_device():
+        # the library launches on the current device
+        raise ValueError(f"tensor is on {t.device}; the current device is cuda:{torch.cuda.current_device()}")
     if not t.is_contiguous():
         raise ValueError("tensor must be contiguous")
     return ctypes.c_void_p(t.data_ptr())

@@ -465,6 +465,8 @@ def run_ours(args):
     cpu = None
     if not args.no_cpu_baseline and world == 1 and rank == 0:
         cpu = cpu_baseline(layers_sample=1)
+        if prefill is not None:
+            prefill["cpu_baseline"] = prefill_cpu_baseline()
 
     # ---- single-matrix HBM gates: each shape at M = 1 over a pool of distinct
     # weight copies (together well beyond L2), as separate launches and as
@@ -774,6 +776,53 @@ def cpu_baseline(layers_sample: int = 1, seconds: float = 10.0):
                             "threads": cores, "ms_per_layer": round(mdt * 1e3 / mreps, 2),
                             "sample": f"{mreps} x the same layer, output rows split over {cores} threads "
                                       f"(sched_getaffinity), {mdt:.1f} s"}
+    return out
+
+
+def prefill_cpu_baseline(seconds: float = 6.0, m_slice: int = 8):
+    """The oracle on the prefill workload (M = 4096, K = 2560, N = 6912,
+    unit RMSNorm gain), timed on an M-slice of m_slice tokens: the oracle's
+    forward costs the same per token, so its TOPS carry over to the full M
+    (reported as extrapolated).  Single-threaded, then with the output rows
+    split over all host cores."""
+    sys.path.insert(0, os.path.join(ROOT, "oracle"))
+    import numpy as np
+
+    import oracle
+    from bitlinear_bitnet_linear_b200 import synthetic
+
+    oracle.build()
+    K, N = 2560, 6912
+    Wq, g = oracle.quant_weights(synthetic.latent_weights(N, K, seed=4242).numpy())
+    x = synthetic.activations(m_slice, K, seed=4243).float().numpy()
+    gain = np.ones(K, np.float32)
+
+    def run(fn, budget):
+        t0 = time.perf_counter()
+        reps = 0
+        while True:
+            fn(x, Wq, g, gain)
+            reps += 1
+            if time.perf_counter() - t0 > budget:
+                break
+        return reps, time.perf_counter() - t0
+
+    ops = 2.0 * m_slice * N * K
+    reps, dt = run(_OracleRows(oracle, 1), seconds)
+    out = {"value": round(ops * reps / dt / 1e12, 6), "unit": "TOPS", "cores": 1, "kind": "oracle",
+           "extrapolated": True,
+           "sample": f"{reps} x an M-slice of {m_slice} tokens of the M = 4096 prefill workload, {dt:.1f} s of "
+                     f"single-threaded scalar C; the per-token cost is constant, so the rate carries over"}
+    cores = host_cores()
+    if cores > 1:
+        many = _OracleRows(oracle, cores)
+        try:
+            mreps, mdt = run(many, seconds / 2)
+        finally:
+            many.close()
+        out["all_cores"] = {"value": round(ops * mreps / mdt / 1e12, 6), "unit": "TOPS", "cores": cores,
+                            "threads": cores, "sample": f"{mreps} x the same slice, output rows split over "
+                                                        f"{cores} threads, {mdt:.1f} s"}
     return out
 
 

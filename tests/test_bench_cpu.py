@@ -124,3 +124,13 @@ def test_hbm_gate_leg_host_logic(monkeypatch):
     n0 = shapes[0]["copies"]
     assert len(set(seen["single"][:n0])) == n0
     assert seen["grouped"] == [e["copies"] for e in shapes for _ in range(2)]
+
+
+def test_prefill_cpu_baseline_line():
+    """The oracle's prefill rate: an M-slice, labelled extrapolated, with the
+    all-cores form when the host has more than one core."""
+    d = bench.prefill_cpu_baseline(seconds=0.3, m_slice=2)
+    assert d["kind"] == "oracle" and d["unit"] == "TOPS" and d["cores"] == 1
+    assert d["extrapolated"] is True and d["value"] > 0
+    if bench.host_cores() > 1:
+        assert d["all_cores"]["cores"] == bench.host_cores() and d["all_cores"]["value"] > 0

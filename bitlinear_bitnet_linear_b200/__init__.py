@@ -12,4 +12,5 @@ from ._binding import (BF16, F32, PATH_AUTO, PATH_GEMV, PATH_TC, BitnetError, bi
                        bitnet_quant_act_relu2, bitnet_quant_weights,
                        bitnet_quant_weights_noalloc, bitnet_quant_weights_workspace_bytes, bitnet_set_wait_limit_us, bitnet_ternarise,
                        bitnet_unpack, bitnet_watchdog_selftest, bitnet_workspace_bytes, bitnet_workspace_init,
+                       bitnet_debug_stream_plan,
                        lib, new_workspace, GroupedCall)

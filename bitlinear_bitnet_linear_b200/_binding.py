@@ -31,7 +31,7 @@ EXPORTS = ("bitnet_workspace_bytes", "bitnet_quant_weights_workspace_bytes", "bi
            "bitnet_linear_grouped_b1", "bitnet_t3_row_bytes", "bitnet_pack_t3", "bitnet_unpack_t3",
            "bitnet_linear_t3", "bitnet_linear_grouped_t3",
            "bitnet_quant_weights_noalloc",
-           "bitnet_set_wait_limit_us", "bitnet_watchdog_selftest")
+           "bitnet_set_wait_limit_us", "bitnet_watchdog_selftest", "bitnet_debug_stream_plan")
 
 
 class GemvProblem(ctypes.Structure):
@@ -90,6 +90,7 @@ def lib() -> ctypes.CDLL:
         "bitnet_linear_grouped": ([P, I32, I64, I32, F, I32, P, SZ, P], I32),
         "bitnet_set_wait_limit_us": ([U32], I32),
         "bitnet_watchdog_selftest": ([P, SZ, U32, P], I32),
+        "bitnet_debug_stream_plan": ([P, P, I32, I64, I32, I32, I32, I32, P, P, P], I32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(L, name)
@@ -175,6 +176,22 @@ def bitnet_set_wait_limit_us(limit_us: int) -> None:
 def bitnet_watchdog_selftest(ws: torch.Tensor, limit_us: int, stream=None) -> None:
     _check(lib().bitnet_watchdog_selftest(_ptr(ws), ws.numel(), int(limit_us), _stream(stream)),
            "bitnet_watchdog_selftest")
+
+
+def bitnet_debug_stream_plan(shapes, M: int, bits: int = 2, prequant: bool = False, sms: int = 148,
+                             smem_optin: int = 232448) -> dict:
+    """The streaming GEMV's plan for problems [(K, N), ...] on a described
+    device (host computation only; no GPU needed)."""
+    n = len(shapes)
+    Ks = (ctypes.c_int64 * n)(*[int(k) for k, _ in shapes])
+    Ns = (ctypes.c_int64 * n)(*[int(v) for _, v in shapes])
+    shape = (ctypes.c_int64 * 5)()
+    rows = (ctypes.c_int32 * n)()
+    task = (ctypes.c_int32 * n)()
+    _check(lib().bitnet_debug_stream_plan(Ks, Ns, n, int(M), int(bits), int(bool(prequant)), int(sms),
+                                          int(smem_optin), shape, rows, task), "bitnet_debug_stream_plan")
+    return {"grid": shape[0], "smem": shape[1], "nxb": shape[2], "nslots": shape[3], "slot_bytes": shape[4],
+            "rows": list(rows), "task": list(task)}
 
 
 # --------------------------------------------------------------------------

@@ -976,6 +976,45 @@ bitnet_status bitnet_watchdog_selftest(void* ws, size_t ws_bytes, uint32_t limit
   return launch_result(cudaSuccess);
 }
 
+// The streaming GEMV's plan for a described device, without touching one.
+bitnet_status bitnet_debug_stream_plan(const int64_t* K, const int64_t* N, int count, int64_t M, int bits,
+                                       int prequant, int sms, int smem_optin, int64_t* shape, int32_t* rows,
+                                       int32_t* task) {
+  if (K == nullptr || N == nullptr) return BITNET_ERR_NULL;
+  if (count < 1 || count > kStreamMaxP || sms < 1 || smem_optin < 1) return BITNET_ERR_SHAPE;
+  if (bits != 1 && bits != 2 && bits != 3) return BITNET_ERR_UNSUPPORTED;
+  std::vector<StreamProblem> sp(count);
+  for (int i = 0; i < count; ++i) {
+    bitnet_status s = check_shape(M, K[i], N[i]);
+    if (s != BITNET_OK) return s;
+    sp[i] = StreamProblem{nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, K[i], N[i]};
+  }
+  DeviceInfo d;
+  d.init = true;
+  d.ok = true;
+  d.sms = sms;
+  d.max_smem_optin = smem_optin;
+  auto* pl = new (std::nothrow) StreamPlan<kStreamMaxP>;
+  if (pl == nullptr) return BITNET_ERR_CUDA;
+  const bitnet_status s = plan_stream<kStreamMaxP>(&d, sp.data(), count, M, BITNET_BF16, prequant != 0, 1e-5f,
+                                                   BITNET_BF16, *pl, bits);
+  if (s == BITNET_OK) {
+    if (shape != nullptr) {
+      shape[0] = pl->grid;
+      shape[1] = pl->smem;
+      shape[2] = pl->p.nxb;
+      shape[3] = pl->p.nslots;
+      shape[4] = pl->p.slot_bytes;
+    }
+    for (int i = 0; i < count; ++i) {
+      if (rows != nullptr) rows[i] = pl->p.prob[i].rc;
+      if (task != nullptr) task[i] = pl->p.prob[i].task;
+    }
+  }
+  delete pl;
+  return s;
+}
+
 // Variant of bitnet_quant_weights that allocates nothing: its scratch is the
 // file-scope array above instead of a caller workspace.
 bitnet_status bitnet_quant_weights_noalloc(const float* W, int64_t N, int64_t K, float eps, int8_t* Wq,

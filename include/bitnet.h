@@ -387,6 +387,32 @@ bitnet_status bitnet_set_wait_limit_us(uint32_t limit_us);
 bitnet_status bitnet_watchdog_selftest(void *ws, size_t ws_bytes, uint32_t limit_us,
                                        bitnet_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Diagnostics.
+ * ------------------------------------------------------------------------ */
+
+/* The launch plan the streaming GEMV (bitnet_linear at small M,
+ * bitnet_linear_grouped, and the b1 and base-3 forms) would use for a
+ * grouped call of `count` problems (1 <= count <= 256) of sizes K[i] x N[i]
+ * with M tokens, on a device described by `sms` (multiprocessor count) and
+ * `smem_optin` (opt-in shared memory per block, bytes).  Pure host
+ * computation: it reads no device and launches nothing, so it also runs
+ * without a GPU.  It is an interface choice of this library; the pages have
+ * no counterpart.
+ *   bits: 2 (bitnet_pack), 1 (bitnet_pack_b1) or 3 (bitnet_pack_t3).
+ *   prequant: nonzero for pre-quantised activations (bitnet_linear_q).
+ *   shape: host array of 5, or NULL: {grid (CTAs), dynamic shared-memory
+ *          bytes per CTA, activation buffers (1 or 2), ring slots per
+ *          consumer warp (1 or 2), bytes per slot}.
+ *   rows, task: host arrays of `count`, or NULL: rows per chunk and the
+ *          contraction task of each problem.
+ * K, N, M follow the library's shape rules (BITNET_ERR_SHAPE otherwise).
+ * Returns BITNET_ERR_UNSUPPORTED when no plan fits the shared memory, which
+ * is when the calls above fall back or fail as their comments say. */
+bitnet_status bitnet_debug_stream_plan(const int64_t *K, const int64_t *N, int count, int64_t M, int bits,
+                                       int prequant, int sms, int smem_optin,
+                                       int64_t *shape, int32_t *rows, int32_t *task);
+
 #ifdef __cplusplus
 }
 #endif

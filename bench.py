@@ -842,8 +842,9 @@ def run_reference(args):
         for (K, N, Wq, g), x in zip(prepared, xs):
             fn(x, Wq, g, gain[K])
 
+    warm = max(3, min(args.warmup, 10))
     try:
-        for _ in range(3):
+        for _ in range(warm):
             step()
         steps = max(1, min(args.steps, 20))
         t0 = time.perf_counter()
@@ -854,7 +855,7 @@ def run_reference(args):
         fn.close()
     v = bytes_sample / dt / 1e9
     return {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
-            "steps": steps, "warmup": 3, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
+            "steps": steps, "warmup": warm, "ms_per_step": round(dt * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8 x ternary -> int32 (scalar C)",
             "data": "synthetic", "config": {"workload": WORKLOAD, "sample": "one layer (7 calls) per step"},
             "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",

@@ -90,3 +90,44 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         bn.bitnet_pack(torch.zeros((4, 16), dtype=torch.int8))
+
+
+def _empty_calls(L):
+    """Each compute entry point with the dimensions it takes: (call, dims)."""
+    F = FAKE
+    z = ctypes.c_size_t(1 << 20)
+    e = 1e-5
+    return {
+        "quant_weights": (lambda M, K, N: L.bitnet_quant_weights(F, N, K, 1e-8, F, F, F, z, None), "KN"),
+        "ternarise": (lambda M, K, N: L.bitnet_ternarise(F, N, K, F, 1e-8, F, None), "KN"),
+        "pack": (lambda M, K, N: L.bitnet_pack(F, N, K, F, None, None), "KN"),
+        "unpack": (lambda M, K, N: L.bitnet_unpack(F, N, K, F, None, None), "KN"),
+        "quant_act": (lambda M, K, N: L.bitnet_quant_act(F, 1, M, K, None, e, F, F, None, None), "MK"),
+        "quant_act_relu2": (lambda M, K, N: L.bitnet_quant_act_relu2(F, F, 1, M, K, None, e, F, F, None, None),
+                            "MK"),
+        "linear": (lambda M, K, N: L.bitnet_linear(F, 1, M, K, F, N, F, None, e, F, 1, F, z, None), "MKN"),
+        "linear_ex": (lambda M, K, N: L.bitnet_linear_ex(F, 1, M, K, F, N, F, None, e, F, 1, F, z, 2, None), "MKN"),
+        "linear_q": (lambda M, K, N: L.bitnet_linear_q(F, F, None, M, K, F, N, F, F, 1, None, F, z, 0, None), "MKN"),
+        "linear_relu2": (lambda M, K, N: L.bitnet_linear_relu2(F, F, 1, M, K, F, N, F, None, e, None, F, 1, F, z,
+                                                               None), "MKN"),
+        "quant_weights_b1": (lambda M, K, N: L.bitnet_quant_weights_b1(F, N, K, F, F, F, z, None), "KN"),
+        "pack_b1": (lambda M, K, N: L.bitnet_pack_b1(F, N, K, F, None, None), "KN"),
+        "unpack_b1": (lambda M, K, N: L.bitnet_unpack_b1(F, N, K, F, None), "KN"),
+        "linear_b1": (lambda M, K, N: L.bitnet_linear_b1(F, 1, M, K, F, N, F, None, e, F, 1, F, z, None), "MKN"),
+        "pack_t3": (lambda M, K, N: L.bitnet_pack_t3(F, N, K, F, None, None), "KN"),
+        "unpack_t3": (lambda M, K, N: L.bitnet_unpack_t3(F, N, K, F, None, None), "KN"),
+        "linear_t3": (lambda M, K, N: L.bitnet_linear_t3(F, 1, K, F, N, F, None, e, F, 1, F, z, None), "KN"),
+        "quant_weights_noalloc": (lambda M, K, N: L.bitnet_quant_weights_noalloc(F, N, K, 1e-8, F, F, None), "KN"),
+    }
+
+
+def test_empty_and_negative_dimensions_rejected(L):
+    """Empty inputs: every compute entry point answers BITNET_ERR_SHAPE for
+    a zero or negative M, K or N it takes, before any device work."""
+    base = {"M": 1, "K": 128, "N": 8}
+    for name, (call, dims) in _empty_calls(L).items():
+        for d in dims:
+            for bad in (0, -16):
+                args = dict(base)
+                args[d] = bad
+                assert call(args["M"], args["K"], args["N"]) == 2, (name, d, bad)

@@ -131,3 +131,13 @@ def test_empty_and_negative_dimensions_rejected(L):
                 args = dict(base)
                 args[d] = bad
                 assert call(args["M"], args["K"], args["N"]) == 2, (name, d, bad)
+
+
+def test_empty_grouped_call_rejected(L):
+    """A grouped call with no problems (or more than 256) is a shape error;
+    the problem table is not read."""
+    z = ctypes.c_size_t(1 << 20)
+    for count in (0, -1, 257):
+        assert L.bitnet_linear_grouped(FAKE, count, 1, 1, 1e-5, 1, FAKE, z, None) == 2
+        assert L.bitnet_linear_grouped_b1(FAKE, count, 1, 1e-5, 1, FAKE, z, None) == 2
+        assert L.bitnet_linear_grouped_t3(FAKE, count, 1, 1e-5, 1, FAKE, z, None) == 2
